@@ -1,0 +1,106 @@
+"""Seeded synthetic workloads shared by the tests, the bench and the smoke run.
+
+This module holds data only: the five segment layouts (text length, image
+grids and frame indices, heads, batch, dtype) and a seeded generator of the
+Q/K/V inputs.  It contains none of the method's arithmetic, so both the CUDA
+path and the float64 oracle may take their inputs from it.
+
+Recipe (the same host arrays feed the oracle and the GPU):
+
+* generator ``numpy.random.default_rng(seed)`` (PCG64);
+* draw order Q, then K, then V, each ``standard_normal((B, L, H, 128))`` in
+  float64, cast to float32, then to bf16 (round-to-nearest-even, via torch)
+  for the bf16 workloads;
+* seeds: tiny 0, t2i 1, edit3 2, maxref 3, hires 4; the max-reference loop's
+  cached steps s = 2..8 draw fresh target Q/K/V with seed 3000 + s;
+* the cached step of the other workloads reuses the target rows of the full
+  step's Q/K/V, so its output must equal the full step's target rows.
+"""
+
+import numpy as np
+import torch
+
+HEAD_DIM = 128
+
+
+def text(n):
+    return {"kind": "text", "n": int(n)}
+
+
+def image(H, W, frame):
+    return {"kind": "image", "H": int(H), "W": int(W), "frame": int(frame)}
+
+
+# Segment layouts of the five workloads: prompt text first, reference images
+# next (frames 1..N), the target image (frame 0) last.
+WORKLOADS = {
+    "tiny": dict(dtype="f32", B=1, H=2, seed=0,
+                 segments=[text(16), image(4, 4, 0)]),
+    "t2i": dict(dtype="bf16", B=1, H=24, seed=1,
+                segments=[text(256), image(64, 64, 0)]),
+    "edit3": dict(dtype="bf16", B=1, H=24, seed=2,
+                  segments=[text(512), image(64, 64, 1), image(64, 64, 2),
+                            image(64, 64, 3), image(64, 64, 0)]),
+    "maxref": dict(dtype="bf16", B=1, H=24, seed=3, cached_steps=7,
+                   segments=[text(1024)] + [image(48, 48, f) for f in range(1, 11)]
+                   + [image(64, 64, 0)]),
+    "hires": dict(dtype="bf16", B=2, H=24, seed=4,
+                  segments=[text(512), image(64, 64, 1), image(128, 128, 0)]),
+}
+
+DESCRIPTIONS = {
+    "tiny": "tiny fp32: B=1, 2 heads, text 16 + target 4x4 (L=32)",
+    "t2i": "text-to-image 1024^2: B=1, 24 heads, text 256 + target 64x64 (L=4352)",
+    "edit3": "edit with 3 references: B=1, 24 heads, text 512 + 3x(64x64) + target 64x64 (L=16896)",
+    "maxref": "max-reference 8-step loop: B=1, 24 heads, text 1024 + 10x(48x48) + target 64x64 (L=28160)",
+    "hires": "high-res 2048^2: B=2, 24 heads, text 512 + ref 64x64 + target 128x128 (L=20992)",
+}
+
+
+def seg_tokens(seg):
+    return seg["n"] if seg["kind"] == "text" else seg["H"] * seg["W"]
+
+
+def sizes(name_or_cfg):
+    """(L, P, T): total tokens, prefix tokens, target tokens (target = last segment)."""
+    cfg = WORKLOADS[name_or_cfg] if isinstance(name_or_cfg, str) else name_or_cfg
+    counts = [seg_tokens(s) for s in cfg["segments"]]
+    L = sum(counts)
+    T = counts[-1]
+    return L, L - T, T
+
+
+def draw_qkv(B, L, H, seed, dtype):
+    """Q, K, V as CPU torch tensors of ``dtype`` ("bf16" or "f32"), [B, L, H, 128]."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(3):
+        x = rng.standard_normal((B, L, H, HEAD_DIM)).astype(np.float32)
+        t = torch.from_numpy(x)
+        out.append(t.to(torch.bfloat16) if dtype == "bf16" else t)
+    return tuple(out)
+
+
+def full_inputs(name):
+    cfg = WORKLOADS[name]
+    L, _, _ = sizes(name)
+    return draw_qkv(cfg["B"], L, cfg["H"], cfg["seed"], cfg["dtype"])
+
+
+def cached_inputs(name, step=2):
+    """Target Q/K/V of a cached step.
+
+    The max-reference loop draws them fresh per step (seed 3000 + step); the
+    other workloads reuse the target rows of the full step's inputs.
+    """
+    cfg = WORKLOADS[name]
+    L, P, T = sizes(name)
+    if name == "maxref":
+        return draw_qkv(cfg["B"], T, cfg["H"], 3000 + step, cfg["dtype"])
+    q, k, v = full_inputs(name)
+    return tuple(x[:, P:].contiguous() for x in (q, k, v))
+
+
+def as_f64(t):
+    """float64 numpy copy of a (CPU) torch tensor, for the oracle."""
+    return t.detach().to("cpu").to(torch.float64).numpy()

@@ -1,0 +1,252 @@
+"""Float64 CPU oracle for the Qwen-Image-2.1 joint-attention hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg (and ``bench.py --impl reference``) may call it.  It shares no code with
+the CUDA library: it is written from the pages' description of the method,
+step by step, with no blocking, fusion or reordering beyond the plain
+definitions.
+
+What it computes (sources are the pages this build follows):
+
+* ``positions`` -- the 3D axial position table and the block-causal visibility
+  bound.  "3A - 3D Axial RoPE (16, 56, 56) & Zero-Centered Grid", section 1
+  (Definition) and the glossary entry "zero-centred grid": text tokens advance
+  frame/height/width together by +1; an image freezes its frame index and
+  numbers rows and columns around (0, 0), height from -(H - H//2) to H//2 - 1
+  (example H = 4 -> -2, -1, 0, 1), width likewise.  Token order inside an image
+  is row-major with width fastest ("Qwen-Image-Edit close reading", section
+  7.3, ``_compute_video_freqs``).  The mask: "Qwen-Image-2.1 architecture"
+  overview, card 3C (text reads only what precedes it, tokens of one image see
+  each other both ways) and the learning goals (the Prefix never attends the
+  target); the target is appended last (card 2A).
+* ``rope_angles`` / ``rope`` -- axial rotary embedding: head_dim 128 split
+  into bands (16, 56, 56) for (frame, height, width) (3A, section 1); per axis
+  the angle of pair j is pos * theta^(-2j/d_axis) with theta = 10000 (close
+  reading, section 7.1: per-axis ``outer(index, 1/theta^(2i/dim))`` turned into
+  unit complex factors by ``torch.polar``), applied to adjacent pairs
+  (2m, 2m+1) as a complex multiplication (close reading, section 6: RoPE on Q
+  and K before attention).
+* ``attention_head`` -- softmax(Q K^T / sqrt(128) + M) V with an explicit
+  dense mask M (0 where key j < kv_end[i], -inf elsewhere); the scale is the
+  SDPA default since the attention call passes none (close reading, section 6).
+* ``prefix_cache`` / ``attn_cached`` -- the Prefix KV Cache: step 1 stores the
+  rotated prefix K and the prefix V; later steps attend the target queries
+  over [cached prefix K/V || fresh target K/V] with no mask, since the target
+  sees everything (overview, card 6A and learning goals).
+
+Inputs are arrays already cast to the GPU dtype (bf16 or fp32) by the seeded
+input module; every function promotes them to float64 first.
+
+Pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
+the pages' worked example, closed forms, invariants and library routines.
+No function is "parity unpinned".
+"""
+
+import math
+
+import numpy as np
+
+HEAD_DIM = 128
+AXES_DIM = (16, 56, 56)  # frame, height, width bands of one head (3A, section 1)
+THETA = 10000.0
+
+
+# ----------------------------------------------------------------------------
+# a1: position table and visibility bound
+# ----------------------------------------------------------------------------
+
+def positions(segments):
+    """Position table ``pos[L, 3]`` = (frame, height, width) and ``kv_end[L]``.
+
+    ``segments`` is the sequence in order; each item is a dict
+    ``{"kind": "text", "n": n}`` or
+    ``{"kind": "image", "H": H, "W": W, "frame": f}``.
+
+    Text: the three coordinates advance together by +1 per text token; the
+    counter starts at 0 and counts text tokens only (3A, section 1).
+    Image: the frame stays fixed over the whole image, the row r and column c
+    (row-major, width fastest) map to h = r - (H - H//2), w = c - (W - W//2)
+    (3A, section 1 and glossary).
+
+    ``kv_end[i]`` is one past the last key token i may attend (block-causal
+    mask, overview card 3C): a text token sees itself and everything before
+    it; an image token sees everything before its image and its whole image.
+    """
+    pos = []
+    kv_end = []
+    text_counter = 0
+    start = 0
+    for seg in segments:
+        if seg["kind"] == "text":
+            n = int(seg["n"])
+            for t in range(n):
+                pos.append((text_counter, text_counter, text_counter))
+                kv_end.append(start + t + 1)
+                text_counter += 1
+            start += n
+        elif seg["kind"] == "image":
+            H, W, frame = int(seg["H"]), int(seg["W"]), int(seg["frame"])
+            end = start + H * W
+            for r in range(H):
+                for c in range(W):
+                    pos.append((frame, r - (H - H // 2), c - (W - W // 2)))
+                    kv_end.append(end)
+            start = end
+        else:
+            raise ValueError("unknown segment kind %r" % (seg["kind"],))
+    return (np.array(pos, dtype=np.int64).reshape(-1, 3),
+            np.array(kv_end, dtype=np.int64))
+
+
+def allowed_matrix(kv_end, n_keys):
+    """Dense boolean mask: allowed[i, j] = j < kv_end[i]."""
+    kv_end = np.asarray(kv_end, dtype=np.int64)
+    return np.arange(n_keys)[None, :] < kv_end[:, None]
+
+
+# ----------------------------------------------------------------------------
+# a2-a4: axial rotary embedding
+# ----------------------------------------------------------------------------
+
+def rope_angles(pos):
+    """Angles ``[L, 64]`` in float64: pair m of the head belongs to one band.
+
+    Pairs 0..7 use the frame axis, 8..35 the height axis, 36..63 the width
+    axis; inside band a of width d_a, pair j turns by pos_a * theta^(-2j/d_a).
+    """
+    pos = np.asarray(pos, dtype=np.int64)
+    L = pos.shape[0]
+    ang = np.empty((L, HEAD_DIM // 2), dtype=np.float64)
+    m = 0
+    for axis, d in enumerate(AXES_DIM):
+        for j in range(d // 2):
+            omega = THETA ** (-2.0 * j / d)
+            ang[:, m] = pos[:, axis].astype(np.float64) * omega
+            m += 1
+    assert m == HEAD_DIM // 2
+    return ang
+
+
+def rope(x, pos):
+    """Rotate ``x[L, 128]`` (one head) by the axial angles of ``pos[L, 3]``.
+
+    Dims (2m, 2m+1) form a complex number x0 + i*x1 that is multiplied by
+    exp(i*phi_m): (x0 cos - x1 sin, x0 sin + x1 cos).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ang = rope_angles(pos)
+    c = np.cos(ang)
+    s = np.sin(ang)
+    x0 = x[:, 0::2]
+    x1 = x[:, 1::2]
+    out = np.empty_like(x)
+    out[:, 0::2] = x0 * c - x1 * s
+    out[:, 1::2] = x0 * s + x1 * c
+    return out
+
+
+# ----------------------------------------------------------------------------
+# a5-a8: masked softmax attention
+# ----------------------------------------------------------------------------
+
+def attention_head(q_rot, k_rot, v, kv_end=None, chunk=512):
+    """softmax(Q K^T / sqrt(128) + M) V for one (batch, head).
+
+    ``q_rot[R,128]`` are the (already rotated) query rows to compute,
+    ``k_rot[Lk,128]`` the rotated keys and ``v[Lk,128]`` the values.
+    ``kv_end[R]`` gives the mask of those rows, M[i, j] = 0 if j < kv_end[i]
+    else -inf; ``None`` means no mask.  The mask is built as an explicit dense
+    matrix for each chunk of rows.
+    """
+    q_rot = np.asarray(q_rot, dtype=np.float64)
+    k_rot = np.asarray(k_rot, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    R = q_rot.shape[0]
+    Lk = k_rot.shape[0]
+    scale = 1.0 / math.sqrt(HEAD_DIM)
+    out = np.empty((R, HEAD_DIM), dtype=np.float64)
+    for c0 in range(0, R, chunk):
+        c1 = min(R, c0 + chunk)
+        S = (q_rot[c0:c1] @ k_rot.T) * scale
+        if kv_end is not None:
+            kv = np.asarray(kv_end, dtype=np.int64)[c0:c1]
+            M = np.where(np.arange(Lk)[None, :] < kv[:, None], 0.0, -np.inf)
+            S = S + M
+        S = S - S.max(axis=1, keepdims=True)
+        E = np.exp(S)
+        out[c0:c1] = (E @ v) / E.sum(axis=1, keepdims=True)
+    return out
+
+
+def attn_full(q, k, v, pos, kv_end, heads=None, rows=None, batches=None):
+    """Full block-causal step for ``q, k, v[B, L, H, 128]``.
+
+    Returns ``o[len(batches), len(rows), len(heads), 128]`` in float64
+    (defaults: all batches, rows and heads).
+    """
+    B, L, H, D = q.shape
+    assert D == HEAD_DIM
+    heads = range(H) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    rows = np.arange(L) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((len(batches), rows.shape[0], len(heads), D), dtype=np.float64)
+    for bi, b in enumerate(batches):
+        for hi, h in enumerate(heads):
+            k_rot = rope(k[b, :, h, :], pos)
+            q_rot = rope(q[b, rows, h, :], np.asarray(pos)[rows])
+            out[bi, :, hi, :] = attention_head(q_rot, k_rot, v[b, :, h, :],
+                                               np.asarray(kv_end)[rows])
+    return out
+
+
+# ----------------------------------------------------------------------------
+# a9: prefix KV cache and the target-only step
+# ----------------------------------------------------------------------------
+
+def prefix_cache(k, v, pos, P, heads=None, batches=None):
+    """Step-1 store: rotated prefix K and prefix V, laid out ``[B, H, P, 128]``."""
+    B, L, H, D = k.shape
+    heads = range(H) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    pos = np.asarray(pos)
+    kc = np.empty((len(batches), len(heads), P, D), dtype=np.float64)
+    vc = np.empty((len(batches), len(heads), P, D), dtype=np.float64)
+    for bi, b in enumerate(batches):
+        for hi, h in enumerate(heads):
+            kc[bi, hi] = rope(k[b, :P, h, :], pos[:P])
+            vc[bi, hi] = np.asarray(v[b, :P, h, :], dtype=np.float64)
+    return kc, vc
+
+
+def attn_cached(q_t, k_t, v_t, pos_t, k_cache, v_cache, heads=None, rows=None, batches=None):
+    """Target-only step: target queries over [cached prefix || target] keys.
+
+    ``q_t, k_t, v_t[B, T, H, 128]``; ``k_cache, v_cache[B, H, P, 128]`` (the
+    cache holds rotated K); no mask.  ``heads``/``batches`` index both the
+    target tensors and the cache (the cache must cover them).
+    """
+    B, T, H, D = q_t.shape
+    heads = range(H) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    pos_t = np.asarray(pos_t)
+    out = np.empty((len(batches), rows.shape[0], len(heads), D), dtype=np.float64)
+    for bi, b in enumerate(batches):
+        for hi, h in enumerate(heads):
+            keys = np.concatenate([np.asarray(k_cache[b, h], dtype=np.float64),
+                                   rope(k_t[b, :, h, :], pos_t)], axis=0)
+            vals = np.concatenate([np.asarray(v_cache[b, h], dtype=np.float64),
+                                   np.asarray(v_t[b, :, h, :], dtype=np.float64)], axis=0)
+            q_rot = rope(q_t[b, rows, h, :], pos_t[rows])
+            out[bi, :, hi, :] = attention_head(q_rot, keys, vals, None)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# measurement helper
+# ----------------------------------------------------------------------------
+
+def allowed_pairs(kv_end):
+    """Number of allowed (query, key) pairs of the full step for one head."""
+    return int(np.sum(np.asarray(kv_end, dtype=np.int64)))

@@ -1,0 +1,381 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+Each ``check_*`` takes the oracle module (or a stand-in with one function
+replaced) so that ``test_mutants_are_caught`` can plant a plausible mistake in
+the oracle and show that at least one pin fails.  Nothing here calls the CUDA
+library.
+"""
+
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as ORACLE
+from oracle import qi21_oracle as OM
+from diffusion_transformer_joint_axial_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _img_rows(O, H, Wd, frame=0, text_before=0):
+    segs = ([W.text(text_before)] if text_before else []) + [W.image(H, Wd, frame)]
+    pos, _ = O.positions(segs)
+    return pos[text_before:].reshape(H, Wd, 3)
+
+
+# ---------------------------------------------------------------- positions --
+
+def check_page_example_h4(O):
+    """3A section 1: H = 4 gives height indices (-2, -1, 0, 1)."""
+    (row,) = _golden_lines("centring_h4.txt")
+    H = int(row[0])
+    expect = [int(x) for x in row[1:]]
+    for Wd in (1, 4, 7):
+        grid = _img_rows(O, H, Wd)
+        assert list(grid[:, 0, 1]) == expect
+        # the same rule numbers the width axis
+        gridT = _img_rows(O, Wd, H)
+        assert list(gridT[0, :, 2]) == expect
+
+
+def check_centring_neg_pos_tables(O):
+    """Close reading 7.3: the centred axis is the last H - H//2 entries of the
+    negative table [-N..-1] followed by the first H//2 entries of [0..N-1]."""
+    N = 64
+    neg = -np.arange(N)[::-1] - 1  # -N, ..., -1
+    posv = np.arange(N)
+    for H in range(1, 10):
+        for Wd in range(1, 10):
+            grid = _img_rows(O, H, Wd, frame=3)
+            exp_h = np.concatenate([neg[N - (H - H // 2):], posv[:H // 2]])
+            exp_w = np.concatenate([neg[N - (Wd - Wd // 2):], posv[:Wd // 2]])
+            # row-major, width fastest: broadcast the axes like view/expand and flatten
+            hh = np.broadcast_to(exp_h[:, None], (H, Wd))
+            ww = np.broadcast_to(exp_w[None, :], (H, Wd))
+            assert np.array_equal(grid[:, :, 1], hh)
+            assert np.array_equal(grid[:, :, 2], ww)
+            assert np.all(grid[:, :, 0] == 3)
+
+
+def check_text_and_frames(O):
+    """3A section 1: text advances all three axes by +1 from 0; an image's
+    frame is frozen at its own index over the whole image."""
+    segs = [W.text(10), W.image(3, 5, 2), W.image(2, 2, 0)]
+    pos, kv_end = O.positions(segs)
+    assert pos.shape == (10 + 15 + 4, 3)
+    assert np.array_equal(pos[:10], np.repeat(np.arange(10)[:, None], 3, axis=1))
+    assert np.all(pos[10:25, 0] == 2) and np.all(pos[25:, 0] == 0)
+
+
+def check_prompt_length_invariance(O):
+    """3A section 4: the same image behind 10 or 30 text tokens gets the same
+    coordinates."""
+    a = _img_rows(O, 6, 8, frame=0, text_before=10)
+    b = _img_rows(O, 6, 8, frame=0, text_before=30)
+    assert np.array_equal(a, b)
+
+
+def check_block_causal_rule(O):
+    """Overview card 3C + learning goals, restated at segment level: a text
+    token reads itself and what precedes it; an image token reads every earlier
+    segment and its own image, never a later segment."""
+    segs = [W.text(3), W.image(2, 2, 1), W.text(2), W.image(2, 3, 0)]
+    sizes = [W.seg_tokens(s) for s in segs]
+    seg_of = np.concatenate([np.full(n, i) for i, n in enumerate(sizes)])
+    L = len(seg_of)
+    brute = np.zeros((L, L), dtype=bool)
+    for i in range(L):
+        for j in range(L):
+            si, sj = seg_of[i], seg_of[j]
+            if segs[si]["kind"] == "text":
+                brute[i, j] = j <= i
+            else:
+                brute[i, j] = sj <= si
+    _, kv_end = O.positions(segs)
+    assert np.array_equal(O.allowed_matrix(kv_end, L), brute)
+
+
+def check_prefix_never_sees_target(O):
+    """Learning goals of the overview: the Prefix never attends the target;
+    the target (appended last) attends everything."""
+    for name in ("t2i", "edit3", "maxref", "hires"):
+        pos, kv_end = O.positions(W.WORKLOADS[name]["segments"])
+        L, P, T = W.sizes(name)
+        assert len(kv_end) == L
+        assert kv_end[:P].max() <= P
+        assert np.all(kv_end[P:] == L)
+
+
+# --------------------------------------------------------------------- rope --
+
+def check_bands(O):
+    rows = {r[0]: [int(x) for x in r[1:]] for r in _golden_lines("bands.txt")}
+    assert tuple(O.AXES_DIM) == tuple(rows["bands"])
+    assert sum(O.AXES_DIM) == rows["head_dim"][0] == O.HEAD_DIM
+    assert [d // 2 for d in O.AXES_DIM] == rows["pairs"]
+
+
+def check_rope_vs_polar(O):
+    """Close reading 7.1: per-axis tables polar(1, outer(index, 1/theta^(2i/dim)))
+    concatenated over the axes, applied as a complex product to adjacent pairs."""
+    rng = np.random.default_rng(11)
+    L = 37
+    pos = np.stack([rng.integers(-20, 20, L), rng.integers(-70, 70, L),
+                    rng.integers(-300, 300, L)], axis=1)
+    x = rng.standard_normal((L, 128))
+    factors = []
+    for axis, dim in enumerate((16, 56, 56)):
+        inv = 1.0 / torch.pow(torch.tensor(10000.0, dtype=torch.float64),
+                              torch.arange(0, dim, 2, dtype=torch.float64) / dim)
+        ang = torch.outer(torch.tensor(pos[:, axis], dtype=torch.float64), inv)
+        factors.append(torch.polar(torch.ones_like(ang), ang))
+    f = torch.cat(factors, dim=1)  # (L, 64) complex
+    xc = torch.view_as_complex(torch.tensor(x).reshape(L, 64, 2))
+    ref = torch.view_as_real(xc * f).reshape(L, 128).numpy()
+    got = O.rope(x, pos)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def check_rope_invariants(O):
+    """3A section 1: rotation, and the product of two rotated vectors depends
+    only on the difference of positions (per axis)."""
+    rng = np.random.default_rng(5)
+    L = 24
+    pos = rng.integers(-50, 50, (L, 3))
+    q = rng.standard_normal((L, 128))
+    k = rng.standard_normal((L, 128))
+    # norm preservation
+    assert np.allclose(np.linalg.norm(O.rope(q, pos), axis=1), np.linalg.norm(q, axis=1), atol=1e-12)
+    # identity at position 0
+    assert np.array_equal(O.rope(q, np.zeros_like(pos)), q)
+    # composition rot(rot(x, p), p') = rot(x, p + p')
+    pos2 = rng.integers(-50, 50, (L, 3))
+    assert np.allclose(O.rope(O.rope(q, pos), pos2), O.rope(q, pos + pos2), atol=1e-10)
+    # relative position: <rot(q,p+c), rot(k,p'+c)> = <rot(q,p), rot(k,p')>
+    posk = rng.integers(-50, 50, (L, 3))
+    c = np.array([7, -13, 29])
+    lhs = O.rope(q, pos + c) @ O.rope(k, posk + c).T
+    rhs = O.rope(q, pos) @ O.rope(k, posk).T
+    assert np.allclose(lhs, rhs, atol=1e-9)
+
+
+# ---------------------------------------------------------------- attention --
+
+def _tiny_problem(seed=3):
+    segs = [W.text(4), W.image(2, 3, 1), W.image(2, 2, 0)]
+    rng = np.random.default_rng(seed)
+    L = 14
+    q, k, v = (rng.standard_normal((1, L, 2, 128)) for _ in range(3))
+    return segs, q, k, v
+
+
+def check_attention_brute_force(O):
+    """Explicit loops over (i, j) with math.exp on a 14-token sequence."""
+    segs, q, k, v = _tiny_problem()
+    pos, kv_end = O.positions(segs)
+    got = O.attn_full(q, k, v, pos, kv_end)
+    L = q.shape[1]
+    for h in range(2):
+        qr = O.rope(q[0, :, h], pos)
+        kr = O.rope(k[0, :, h], pos)
+        for i in range(L):
+            logits = [sum(qr[i, d] * kr[j, d] for d in range(128)) / math.sqrt(128)
+                      for j in range(int(kv_end[i]))]
+            mx = max(logits)
+            w = [math.exp(s - mx) for s in logits]
+            tot = sum(w)
+            o = [sum(w[j] * v[0, j, h, d] for j in range(len(w))) / tot for d in range(128)]
+            assert np.max(np.abs(np.array(o) - got[0, i, h])) < 1e-12
+
+
+def check_attention_closed_forms(O):
+    segs, q, k, v = _tiny_problem()
+    pos, kv_end = O.positions(segs)
+    # Q = 0: every logit is 0, so O_i is the mean of the allowed V_j
+    got = O.attn_full(np.zeros_like(q), k, v, pos, kv_end)
+    for i in range(q.shape[1]):
+        assert np.allclose(got[0, i], v[0, :kv_end[i]].mean(axis=0), atol=1e-13)
+    # constant V along keys: O = V
+    vc = np.broadcast_to(v[:, :1], v.shape).copy()
+    assert np.allclose(O.attn_full(q, k, vc, pos, kv_end), vc, atol=1e-13)
+    # the first text token sees only itself: O_0 = V_0 exactly
+    assert np.array_equal(O.attn_full(q, k, v, pos, kv_end)[0, 0], v[0, 0])
+
+
+def check_attention_vs_sdpa(O):
+    """With no mask and every position 0 the method is plain softmax attention:
+    torch's scaled_dot_product_attention in float64 must agree."""
+    rng = np.random.default_rng(9)
+    L = 40
+    q, k, v = (rng.standard_normal((1, L, 3, 128)) for _ in range(3))
+    pos = np.zeros((L, 3), dtype=np.int64)
+    kv_end = np.full(L, L)
+    got = O.attn_full(q, k, v, pos, kv_end)
+    tq, tk, tv = (torch.tensor(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(got - ref)) < 1e-12
+    # and with the block-causal mask handed to SDPA as a boolean mask
+    segs, q2, k2, v2 = _tiny_problem(4)
+    pos2, kv2 = O.positions(segs)
+    got2 = O.attn_full(q2, k2, v2, np.zeros_like(pos2), kv2)
+    allowed = torch.tensor(O.allowed_matrix(kv2, q2.shape[1]))
+    tq, tk, tv = (torch.tensor(x).permute(0, 2, 1, 3) for x in (q2, k2, v2))
+    ref2 = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed)
+    assert np.max(np.abs(got2 - ref2.permute(0, 2, 1, 3).numpy())) < 1e-12
+
+
+def check_prefix_invariance(O):
+    """Learning goals: the Prefix never attends the target, so perturbing the
+    target's Q/K/V leaves every prefix output unchanged."""
+    segs, q, k, v = _tiny_problem()
+    pos, kv_end = O.positions(segs)
+    P = 10
+    base = O.attn_full(q, k, v, pos, kv_end)
+    rng = np.random.default_rng(1)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for x in (q2, k2, v2):
+        x[:, P:] += rng.standard_normal(x[:, P:].shape)
+    pert = O.attn_full(q2, k2, v2, pos, kv_end)
+    assert np.array_equal(base[:, :P], pert[:, :P])
+    assert not np.allclose(base[:, P:], pert[:, P:])
+
+
+def check_cached_equals_full(O):
+    """Overview (lab note): reusing the Prefix K/V reproduces the full
+    recomputation to float64 rounding."""
+    segs, q, k, v = _tiny_problem()
+    pos, kv_end = O.positions(segs)
+    P = 10
+    full = O.attn_full(q, k, v, pos, kv_end)
+    kc, vc = O.prefix_cache(k, v, pos, P)
+    assert np.array_equal(vc, np.transpose(v[:, :P], (0, 2, 1, 3)))
+    cached = O.attn_cached(q[:, P:], k[:, P:], v[:, P:], pos[P:], kc, vc)
+    assert np.max(np.abs(cached - full[:, P:])) < 1e-13
+
+
+CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_frames,
+          check_prompt_length_invariance, check_block_causal_rule, check_prefix_never_sees_target,
+          check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
+          check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
+          check_cached_equals_full]
+
+
+@pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
+def test_oracle_pin(check):
+    check(ORACLE)
+
+
+# ------------------------------------------------------------------ mutants --
+
+def _mutant(**repl):
+    ns = types.SimpleNamespace(**{k: getattr(OM, k) for k in dir(OM) if not k.startswith("_")})
+    for k, fn in repl.items():
+        setattr(ns, k, fn)
+    # rebind the helpers that call each other so the mutation propagates
+    def attn_full(q, k, v, pos, kv_end, heads=None, rows=None, batches=None):
+        B, L, H, D = q.shape
+        out = np.empty((B, L, H, D))
+        for b in range(B):
+            for h in range(H):
+                out[b, :, h] = ns.attention_head(ns.rope(q[b, :, h], pos), ns.rope(k[b, :, h], pos),
+                                                 v[b, :, h], kv_end)
+        return out
+    if "attn_full" not in repl:
+        ns.attn_full = attn_full
+    return ns
+
+
+def _rope_sign_flipped(x, pos):
+    out = OM.rope(x, pos)
+    ref = np.asarray(x, dtype=np.float64)
+    return 2 * ref * np.cos(OM.rope_angles(pos)).repeat(2, axis=1) - out
+
+
+def _angles_global_denominator(pos):
+    pos = np.asarray(pos)
+    ang = np.empty((pos.shape[0], 64))
+    m = 0
+    for axis, d in enumerate(OM.AXES_DIM):
+        for j in range(d // 2):
+            ang[:, m] = pos[:, axis] * OM.THETA ** (-2.0 * j / 128)
+            m += 1
+    return ang
+
+
+def _rope_with(angles_fn):
+    def rope(x, pos):
+        x = np.asarray(x, dtype=np.float64)
+        a = angles_fn(pos)
+        c, s = np.cos(a), np.sin(a)
+        out = np.empty_like(x)
+        out[:, 0::2] = x[:, 0::2] * c - x[:, 1::2] * s
+        out[:, 1::2] = x[:, 0::2] * s + x[:, 1::2] * c
+        return out
+    return rope
+
+
+def _positions_floor_centre(segs):
+    pos, kv_end = OM.positions(segs)
+    start = 0
+    for s in segs:
+        n = W.seg_tokens(s)
+        if s["kind"] == "image":
+            H, Wd = s["H"], s["W"]
+            r = np.arange(n) // Wd
+            c = np.arange(n) % Wd
+            pos[start:start + n, 1] = r - H // 2
+            pos[start:start + n, 2] = c - Wd // 2
+        start += n
+    return pos, kv_end
+
+
+def _positions_text_exclusive(segs):
+    pos, kv_end = OM.positions(segs)
+    start = 0
+    for s in segs:
+        n = W.seg_tokens(s)
+        if s["kind"] == "text":
+            kv_end[start:start + n] -= 1
+        start += n
+    return pos, kv_end
+
+
+def _head_no_scale(q_rot, k_rot, v, kv_end=None, chunk=512):
+    return OM.attention_head(q_rot * math.sqrt(128), k_rot, v, kv_end, chunk)
+
+
+def _head_v_transposed(q_rot, k_rot, v, kv_end=None, chunk=512):
+    return OM.attention_head(q_rot, k_rot, v[::-1], kv_end, chunk)
+
+
+MUTANTS = {
+    "rope_sign": dict(rope=_rope_sign_flipped),
+    "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
+                                 rope_angles=_angles_global_denominator),
+    "centre_floor": dict(positions=_positions_floor_centre),
+    "text_mask_exclusive": dict(positions=_positions_text_exclusive),
+    "missing_scale": dict(attention_head=_head_no_scale),
+    "value_order": dict(attention_head=_head_v_transposed),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutants_are_caught(name):
+    ns = _mutant(**MUTANTS[name])
+    failed = []
+    for check in CHECKS:
+        try:
+            with np.errstate(all="ignore"):
+                check(ns)
+        except (AssertionError, ValueError, IndexError, FloatingPointError):
+            failed.append(check.__name__)
+    assert failed, "planted mistake %s passed every pin" % name
