@@ -1,0 +1,369 @@
+"""Benchmark of the Qwen-Image-2.1 joint-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+position table -> full block-causal step (axial RoPE, tile-skipping mask,
+Prefix KV cache store) -> one prefix-cached target-only step.  The metric is
+algorithmic TFLOP/s: 4 * 128 * (allowed query/key pairs) per (batch, head),
+masked tiles and elements excluded.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload t2i]
+    python bench.py --impl reference ...   # the float64 CPU oracle, timed
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own copy of the
+workload (independent requests; no data exchange), the device time is the max
+over ranks and ``value`` is the work of all ranks over that time (weak scaling).
+Prints one JSON line on rank 0.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from diffusion_transformer_joint_axial_b200 import workloads as W  # noqa: E402
+
+METRIC = "joint-attn TFLOP/s (full step & prefix-cached step), % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers --
+
+def step_flops(name):
+    """Algorithmic FLOPs of one step: full step + one cached step, all heads."""
+    cfg = W.WORKLOADS[name]
+    L, P, T = W.sizes(name)
+    # allowed pairs of the full step: sum over rows of their visibility bound
+    # (the segment layout fixes it: text token i sees i + 1 keys, an image
+    # token sees everything up to the end of its image)
+    pairs = 0
+    start = 0
+    for s in cfg["segments"]:
+        n = W.seg_tokens(s)
+        if s["kind"] == "text":
+            pairs += n * start + n * (n + 1) // 2
+        else:
+            pairs += n * (start + n)
+        start += n
+    full = 4.0 * 128 * pairs * cfg["B"] * cfg["H"]
+    cached = 4.0 * 128 * T * (P + T) * cfg["B"] * cfg["H"]
+    return full, cached
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            backend="nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device):
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle --
+
+def oracle_sample(name, budget_s):
+    """Times the float64 oracle on a bounded sample of the workload: whole
+    heads of the full step and of one cached step, until ``budget_s`` passes.
+    Returns (flops, seconds, heads done)."""
+    import oracle as O
+    cfg = W.WORKLOADS[name]
+    L, P, T = W.sizes(name)
+    q, k, v = W.draw_qkv(1, L, 1, cfg["seed"], cfg["dtype"])
+    qf, kf, vf = W.as_f64(q), W.as_f64(k), W.as_f64(v)
+    pos, kv_end = O.positions(cfg["segments"])
+    full1, cached1 = (x / (cfg["B"] * cfg["H"]) for x in step_flops(name))
+    flops, heads = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        O.attn_full(qf, kf, vf, pos, kv_end)
+        kc, vc = O.prefix_cache(kf, vf, pos, P)
+        O.attn_cached(qf[:, P:], kf[:, P:], vf[:, P:], pos[P:], kc, vc)
+        flops += full1 + cached1
+        heads += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or heads >= cfg["B"] * cfg["H"]:
+            return flops, dt, heads
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    name = args.workload
+    cfg = W.WORKLOADS[name]
+    for _ in range(args.warmup):
+        oracle_sample(name, 0.0)
+    tot_f, tot_s, heads = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        f, s, h = oracle_sample(name, 0.0)
+        tot_f, tot_s, heads = tot_f + f, tot_s + s, heads + h
+    value = tot_f / tot_s / 1e12
+    sample = "%d head(s) of the %s full step + one cached step per bench step (float64 oracle, %s)" % (
+        heads // max(1, args.steps), name, W.DESCRIPTIONS[name])
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": W.DESCRIPTIONS[name], "B": cfg["B"], "H": cfg["H"]},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm --
+
+def run_ours(args, world, rank, local):
+    import diffusion_transformer_joint_axial_b200 as qi
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    cfg = W.WORKLOADS[name]
+    assert cfg["dtype"] == "bf16", "the bench measures the bf16 workloads"
+    B, H = cfg["B"], cfg["H"]
+    L, P, T = W.sizes(name)
+    segs = cfg["segments"]
+    dt = torch.bfloat16
+
+    # inputs (host, pinned) and device-resident copies
+    q, k, v = W.full_inputs(name)
+    qt, kt, vt = W.cached_inputs(name, 2)
+    host = [x.pin_memory() for x in (q, k, v, qt, kt, vt)]
+    dq, dk, dv, dqt, dkt, dvt = (x.to(dev) for x in host)
+    kc, vc = qi.alloc_cache(B, H, P, dt, dev)
+    o_full = torch.empty_like(dq)
+    o_c = torch.empty_like(dqt)
+    ws_f = qi.new_workspace(qi.full_workspace_size(B, H, L, P, dt), dev)
+    ws_c = qi.new_workspace(qi.cached_workspace_size(B, H, P, T, dt), dev)
+    pos = torch.empty((L, 3), dtype=torch.int32, device=dev)
+    kv_end = torch.empty((L,), dtype=torch.int32, device=dev)
+    seg_arr = qi._binding.to_segments(segs)
+    lib = qi.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sp = qi._binding.ctypes.c_void_p(stream.cuda_stream)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    P_ = qi._binding._ptr
+
+    def one_step(ev=None, qq=dq, kk=dk, vv=dv, qqt=dqt, kkt=dkt, vvt=dvt):
+        lib.qi21_rope_positions(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
+        if ev is not None:
+            qi.time_next_attention(ev[0], ev[1])
+        st = lib.qi21_attn_full(B, H, L, P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
+                                P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
+        assert st == 0, lib.qi21_last_error()
+        if ev is not None:
+            qi.time_next_attention(ev[2], ev[3])
+        st = lib.qi21_attn_cached(B, H, P, T, 0, P_(qqt), P_(kkt), P_(vvt), P_(pos[P:]), P_(kc), P_(vc),
+                                  P_(o_c), P_(ws_c), ws_c.numel(), sp)
+        assert st == 0, lib.qi21_last_error()
+
+    full_flops, cached_flops = step_flops(name)
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
+
+    # ---- device-resident timing
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [(mk(), mk(), mk(), mk(), mk(), mk()) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if rank == 0 else None
+    n0 = qi.launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        e = evs[i]
+        e[4].record(stream)
+        one_step(ev=e)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = qi.launch_count() - n0
+    clk = clocks.stop() if clocks else None
+    step_ms = sum(e[4].elapsed_time(e[5]) for e in evs)
+    full_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    cached_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
+
+    # ---- end to end through the C ABI with host buffers (copies timed)
+    h2d = sum(x.numel() * x.element_size() for x in host)
+    d2h = (o_full.numel() + o_c.numel()) * 2
+    out_h = [torch.empty(o_full.shape, dtype=dt, pin_memory=True),
+             torch.empty(o_c.shape, dtype=dt, pin_memory=True)]
+    e2e_steps = max(3, min(args.steps, 20))
+    ee = [(mk(), mk()) for _ in range(e2e_steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        ee[i][0].record(stream)
+        for d, h in zip((dq, dk, dv, dqt, dkt, dvt), host):
+            d.copy_(h, non_blocking=True)
+        one_step()
+        out_h[0].copy_(o_full, non_blocking=True)
+        out_h[1].copy_(o_c, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
+
+    tot_flops = (full_flops + cached_flops) * args.steps
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
+    all_flops = sum_over_ranks(tot_flops, world, dev)
+    all_e2e_flops = sum_over_ranks((full_flops + cached_flops) * e2e_steps, world, dev)
+    value = all_flops / (step_ms_max * 1e-3) / 1e12
+    e2e_value = all_e2e_flops / (e2e_ms_max * 1e-3) / 1e12
+    if rank != 0:
+        return
+
+    peaks, kind = load_peaks()
+    peak = peaks["bf16_tflops"]
+    att_ms = full_ms + cached_ms
+    achieved = (full_flops + cached_flops) * args.steps / (att_ms * 1e-3) / 1e12
+    full_tf = full_flops * args.steps / (full_ms * 1e-3) / 1e12
+    cached_tf = cached_flops * args.steps / (cached_ms * 1e-3) / 1e12
+
+    budget = 0.0 if args.no_cpu_baseline else args.cpu_budget
+    cpu = None
+    if budget > 0:
+        f, s, heads = oracle_sample(name, budget)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": "%d of %d (batch, head) pairs of the %s step (full + one cached), float64 "
+                         "NumPy oracle, %.1f s" % (heads, B * H, name, s)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": W.DESCRIPTIONS[name], "B": B, "H": H, "L": L, "P": P, "T": T,
+                   "step": "positions + full block-causal step with cache store + one cached step",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "parallelism": "dp%d (independent requests per GPU)" % world},
+        "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps},
+        "cached_step": {"tflops": cached_tf, "frac_of_peak": cached_tf / peak,
+                        "ms": cached_ms / args.steps},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "qi21::tc::attn_tc_kernel (full + cached launches)",
+                     "peak_kind": "%s bf16 dense burst (cuBLAS), MEASURED_PEAKS.json" % kind},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="t2i", choices=[n for n in W.WORKLOADS if n != "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,16 @@
+"""Qwen-Image-2.1 joint-attention hot path for B200 (sm_100a).
+
+3D axial RoPE (bands 16/56/56, centred image grids), the Block-Causal mask
+and the Prefix KV Cache, computed by the CUDA kernels of ``libqi21.so``
+behind a C ABI (``include/qi21.h``).  This package is the thin Python
+binding: it marshals torch tensors into that ABI and nothing else.
+"""
+
+from ._binding import (QI21Error, Segment, alloc_cache, attn_cached, attn_full, cached_workspace_size,
+                       full_workspace_size, launch_count, load_library, new_workspace, rope_positions,
+                       selftest_wait_timeout, time_next_attention, workspace_status, HEAD_DIM,
+                       LIB_PATH)
+
+__all__ = ["QI21Error", "Segment", "alloc_cache", "attn_cached", "attn_full", "cached_workspace_size",
+           "full_workspace_size", "launch_count", "load_library", "new_workspace", "rope_positions",
+           "selftest_wait_timeout", "time_next_attention", "workspace_status", "HEAD_DIM", "LIB_PATH"]

@@ -1,0 +1,260 @@
+"""ctypes binding of libqi21 (argument marshalling only).
+
+Every step of the path runs in the library's CUDA kernels; torch supplies
+device memory and the current stream.  If ``libqi21.so`` is missing or no
+CUDA device is present, every call raises ``QI21Error``: there is no fallback.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqi21.so")
+
+QI21_OK = 0
+QI21_ERR_INVALID_ARG = 1
+QI21_ERR_UNSUPPORTED = 2
+QI21_ERR_CUDA = 3
+QI21_ERR_TIMEOUT = 4
+QI21_BF16 = 0
+QI21_F32 = 1
+HEAD_DIM = 128
+MAX_SEGMENTS = 128
+WORKSPACE_HEADER_BYTES = 256
+
+EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_full",
+            "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
+            "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
+            "qi21_launch_count", "qi21_time_next_attention")
+
+
+class QI21Error(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(message)
+        self.status = status
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("n", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("W", ctypes.c_int32), ("frame", ctypes.c_int32)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+
+
+def load_library(path=LIB_PATH):
+    """Loads libqi21.so and declares its C signatures (no CUDA needed)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise QI21Error(QI21_ERR_UNSUPPORTED,
+                        "libqi21.so is not built (python -m diffusion_transformer_joint_axial_b200.build)")
+    L = ctypes.CDLL(path)
+    L.qi21_rope_positions.argtypes = [ctypes.POINTER(Segment), _i32, _i64, _vp, _vp, _vp]
+    L.qi21_attn_full_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i32]
+    L.qi21_attn_full_workspace_size.restype = _sz
+    L.qi21_attn_full.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _sz, _vp]
+    L.qi21_attn_cached_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i32]
+    L.qi21_attn_cached_workspace_size.restype = _sz
+    L.qi21_attn_cached.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _sz, _vp]
+    L.qi21_workspace_status.argtypes = [_vp, _vp]
+    L.qi21_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
+    L.qi21_status_string.argtypes = [_i32]
+    L.qi21_status_string.restype = ctypes.c_char_p
+    L.qi21_last_error.argtypes = []
+    L.qi21_last_error.restype = ctypes.c_char_p
+    L.qi21_launch_count.argtypes = []
+    L.qi21_launch_count.restype = ctypes.c_uint64
+    L.qi21_time_next_attention.argtypes = [_vp, _vp]
+    L.qi21_time_next_attention.restype = None
+    for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached",
+                 "qi21_workspace_status", "qi21_selftest_wait_timeout"):
+        getattr(L, name).restype = _i32
+    _lib = L
+    return L
+
+
+def _check(status):
+    if status != QI21_OK:
+        L = load_library()
+        raise QI21Error(status, "%s: %s" % (L.qi21_status_string(status).decode(),
+                                            L.qi21_last_error().decode()))
+
+
+def _cuda_lib():
+    if not torch.cuda.is_available():
+        raise QI21Error(QI21_ERR_CUDA, "libqi21 needs a CUDA device; none is available")
+    return load_library()
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return QI21_BF16
+    if t.dtype == torch.float32:
+        return QI21_F32
+    raise QI21Error(QI21_ERR_UNSUPPORTED, "dtype %s is not supported (bf16 or fp32)" % t.dtype)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t, name, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise QI21Error(QI21_ERR_INVALID_ARG, "%s must be a torch.Tensor" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise QI21Error(QI21_ERR_INVALID_ARG, "%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype != dtype or t.device != device or not t.is_contiguous():
+        raise QI21Error(QI21_ERR_INVALID_ARG,
+                        "%s must be a contiguous %s tensor on %s" % (name, dtype, device))
+
+
+def to_segments(segments):
+    """ctypes array from dicts {"kind": "text", "n"} / {"kind": "image", "H", "W", "frame"}."""
+    arr = (Segment * max(1, len(segments)))()
+    for i, s in enumerate(segments):
+        if s["kind"] == "text":
+            arr[i] = Segment(0, int(s["n"]), 0, 0, 0)
+        elif s["kind"] == "image":
+            arr[i] = Segment(1, 0, int(s["H"]), int(s["W"]), int(s["frame"]))
+        else:
+            raise QI21Error(QI21_ERR_INVALID_ARG, "unknown segment kind %r" % (s["kind"],))
+    return arr
+
+
+def rope_positions(segments, device="cuda", with_kv_end=True):
+    """Position table ``pos[L, 3]`` (int32) and ``kv_end[L]`` on ``device``."""
+    L_ = _cuda_lib()
+    device = torch.device(device)
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    segs = to_segments(segments)
+    n = sum(int(s["n"]) if s["kind"] == "text" else int(s["H"]) * int(s["W"]) for s in segments)
+    pos = torch.empty((n, 3), dtype=torch.int32, device=device)
+    kv_end = torch.empty((n,), dtype=torch.int32, device=device) if with_kv_end else None
+    with torch.cuda.device(device):
+        _check(L_.qi21_rope_positions(segs, len(segments), n, _ptr(pos), _ptr(kv_end), _stream(device)))
+    return pos, kv_end
+
+
+def full_workspace_size(B, H, L, P, dtype):
+    code = QI21_BF16 if dtype == torch.bfloat16 else QI21_F32
+    return int(load_library().qi21_attn_full_workspace_size(B, H, L, P, code))
+
+
+def cached_workspace_size(B, H, P, T, dtype):
+    code = QI21_BF16 if dtype == torch.bfloat16 else QI21_F32
+    return int(load_library().qi21_attn_cached_workspace_size(B, H, P, T, code))
+
+
+def new_workspace(nbytes, device):
+    """Zeroed device workspace (the header must start at zero)."""
+    return torch.zeros(max(int(nbytes), WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def alloc_cache(B, H, P, dtype, device):
+    """Empty Prefix KV cache pair, [B, H, P, 128] each."""
+    return (torch.empty((B, H, P, HEAD_DIM), dtype=dtype, device=device),
+            torch.empty((B, H, P, HEAD_DIM), dtype=dtype, device=device))
+
+
+def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=None, workspace=None):
+    """First step: block-causal joint attention; stores the prefix K/V cache if given.
+
+    q, k, v: [B, L, H, 128] bf16 or fp32 on one CUDA device; pos [L, 3],
+    kv_end [L] int32 from :func:`rope_positions`.  Returns ``out``.
+    """
+    L_ = _cuda_lib()
+    B, L, H, D = q.shape
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, (B, L, H, HEAD_DIM), dt, dev)
+    _need(pos, "pos", (L, 3), torch.int32, dev)
+    _need(kv_end, "kv_end", (L,), torch.int32, dev)
+    P = int(prefix_len)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", (B, L, H, HEAD_DIM), dt, dev)
+    if (k_cache is None) != (v_cache is None):
+        raise QI21Error(QI21_ERR_INVALID_ARG, "give both k_cache and v_cache or neither")
+    if k_cache is not None:
+        _need(k_cache, "k_cache", (B, H, P, HEAD_DIM), dt, dev)
+        _need(v_cache, "v_cache", (B, H, P, HEAD_DIM), dt, dev)
+    need = full_workspace_size(B, H, L, P, dt)
+    if workspace is None:
+        workspace = new_workspace(need, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_attn_full(B, H, L, P, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(kv_end),
+                                 _ptr(out), _ptr(k_cache), _ptr(v_cache), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(dev)))
+    return out
+
+
+def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None):
+    """Later step: target queries over [cached prefix K/V || fresh target K/V], no mask.
+
+    q, k, v: [B, T, H, 128]; pos_tgt [T, 3]; k_cache, v_cache [B, H, P, 128].
+    """
+    L_ = _cuda_lib()
+    B, T, H, D = q.shape
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, (B, T, H, HEAD_DIM), dt, dev)
+    _need(pos_tgt, "pos_tgt", (T, 3), torch.int32, dev)
+    P = k_cache.shape[2]
+    _need(k_cache, "k_cache", (B, H, P, HEAD_DIM), dt, dev)
+    _need(v_cache, "v_cache", (B, H, P, HEAD_DIM), dt, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", (B, T, H, HEAD_DIM), dt, dev)
+    need = cached_workspace_size(B, H, P, T, dt)
+    if workspace is None:
+        workspace = new_workspace(need, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_attn_cached(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_tgt),
+                                   _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(dev)))
+    return out
+
+
+def workspace_status(workspace):
+    """Synchronises the current stream and returns (and clears) the status word."""
+    L_ = _cuda_lib()
+    with torch.cuda.device(workspace.device):
+        return int(L_.qi21_workspace_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def selftest_wait_timeout(workspace, limit_ns):
+    L_ = _cuda_lib()
+    with torch.cuda.device(workspace.device):
+        _check(L_.qi21_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(workspace.device)))
+
+
+def launch_count():
+    """Kernel launches this thread has enqueued through libqi21."""
+    return int(load_library().qi21_launch_count())
+
+
+def time_next_attention(start, stop):
+    """Brackets the next attention-kernel launch with two torch CUDA events
+    (recorded on the kernel's own launch stream)."""
+    for e in (start, stop):
+        if e.cuda_event == 0:
+            e.record()  # torch creates the event lazily on first record
+    load_library().qi21_time_next_attention(ctypes.c_void_p(start.cuda_event),
+                                             ctypes.c_void_p(stop.cuda_event))

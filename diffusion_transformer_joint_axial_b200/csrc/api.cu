@@ -1,0 +1,328 @@
+// Host side of the libqi21 C ABI (include/qi21.h): argument validation,
+// workspace carving, and the kernel sequence of each entry point.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/qi21.h"
+#include "qi21_internal.h"
+
+namespace qi21 {
+
+static thread_local char g_last_error[512] = "";
+static thread_local uint64_t g_launches = 0;
+static thread_local cudaEvent_t g_time_start = nullptr, g_time_stop = nullptr;
+
+void note_launch() { ++g_launches; }
+
+static qi21_status fail(qi21_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+static qi21_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(QI21_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static size_t elem_bytes(qi21_dtype dt) { return dt == QI21_F32 ? 4 : 2; }
+
+// Workspace: [header][cos/sin table: rows x 64 float2][rotated K: B x H x rows x 128]
+struct WsLayout {
+  size_t table_off, k_off, total;
+};
+static WsLayout ws_layout(int64_t B, int64_t H, int64_t rows, qi21_dtype dt) {
+  WsLayout w;
+  w.table_off = QI21_WORKSPACE_HEADER_BYTES;
+  w.k_off = round_up(w.table_off + (size_t)rows * kPairs * sizeof(float2), 256);
+  w.total = round_up(w.k_off + (size_t)B * H * rows * kHeadDim * elem_bytes(dt), 256);
+  return w;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+static qi21_status check_common(int32_t B, int32_t H, qi21_dtype dt) {
+  if (B < 0 || H < 0) return fail(QI21_ERR_INVALID_ARG, "B and H must be >= 0 (got %d, %d)", B, H);
+  if (dt != QI21_BF16 && dt != QI21_F32) return fail(QI21_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+  return QI21_OK;
+}
+
+static qi21_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(QI21_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(QI21_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return QI21_OK;
+}
+
+#define QI21_TRY(x)                        \
+  do {                                     \
+    qi21_status _s = (x);                  \
+    if (_s != QI21_OK) return _s;          \
+  } while (0)
+
+// Runs the attention kernel that matches the dtype.
+static qi21_status run_attention(const AttnArgs& a, qi21_dtype dt, cudaStream_t st) {
+  cudaEvent_t t0 = g_time_start, t1 = g_time_stop;
+  g_time_start = g_time_stop = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (t0 != nullptr && t1 != nullptr) e = cudaEventRecord(t0, st);
+  if (e == cudaSuccess)
+    e = dt == QI21_F32 ? launch_attn_simt_f32(a, st) : launch_attn_tc_bf16(a, st, sm_count());
+  if (e == cudaSuccess && t0 != nullptr && t1 != nullptr) e = cudaEventRecord(t1, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return QI21_OK;
+}
+
+}  // namespace qi21
+
+using namespace qi21;
+
+extern "C" {
+
+qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_t L, int32_t* pos,
+                                int32_t* kv_end, void* stream) {
+  if (n_segs == 0 && L == 0) return QI21_OK;
+  if (segs == nullptr) return fail(QI21_ERR_INVALID_ARG, "segs is NULL");
+  if (n_segs < 1 || n_segs > QI21_MAX_SEGMENTS)
+    return fail(QI21_ERR_INVALID_ARG, "n_segs must be in [1, %d] (got %d)", QI21_MAX_SEGMENTS, n_segs);
+  if (pos == nullptr) return fail(QI21_ERR_INVALID_ARG, "pos is NULL");
+  PositionsParams p;
+  memset(&p, 0, sizeof(p));
+  int64_t start = 0, text = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const qi21_segment& s = segs[i];
+    int64_t n;
+    if (s.kind == QI21_SEG_TEXT) {
+      if (s.n < 1) return fail(QI21_ERR_INVALID_ARG, "segment %d: text needs n >= 1", i);
+      n = s.n;
+    } else if (s.kind == QI21_SEG_IMAGE) {
+      if (s.H < 1 || s.W < 1) return fail(QI21_ERR_INVALID_ARG, "segment %d: image needs H, W >= 1", i);
+      n = (int64_t)s.H * s.W;
+    } else {
+      return fail(QI21_ERR_INVALID_ARG, "segment %d: unknown kind %d", i, s.kind);
+    }
+    p.segs[i].kind = s.kind;
+    p.segs[i].n = s.n;
+    p.segs[i].H = s.H;
+    p.segs[i].W = s.W;
+    p.segs[i].frame = s.frame;
+    p.segs[i].start = (int32_t)start;
+    p.segs[i].text_base = (int32_t)text;
+    if (s.kind == QI21_SEG_TEXT) text += n;
+    start += n;
+    if (start > INT32_MAX / 2) return fail(QI21_ERR_INVALID_ARG, "sequence too long");
+  }
+  if (start != L) return fail(QI21_ERR_INVALID_ARG, "segments hold %lld tokens, L = %lld", (long long)start, (long long)L);
+  p.n_segs = n_segs;
+  p.L = L;
+  p.pos = pos;
+  p.kv_end = kv_end;
+  cudaError_t e = launch_positions(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions launch");
+  return QI21_OK;
+}
+
+size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt) {
+  (void)P;
+  if (B < 0 || H < 0 || L < 0) return 0;
+  return ws_layout(B, H, L, dt).total;
+}
+
+size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt) {
+  (void)P;
+  if (B < 0 || H < 0 || T < 0) return 0;
+  return ws_layout(B, H, T, dt).total;
+}
+
+qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt, const void* q,
+                           const void* k, const void* v, const int32_t* pos, const int32_t* kv_end,
+                           void* o, void* k_cache, void* v_cache, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  QI21_TRY(check_common(B, H, dt));
+  if (L < 0 || L > (int64_t)1 << 30) return fail(QI21_ERR_INVALID_ARG, "L out of range (%lld)", (long long)L);
+  if (P < 0 || P > L) return fail(QI21_ERR_INVALID_ARG, "P must be in [0, L] (P=%lld, L=%lld)", (long long)P, (long long)L);
+  if ((k_cache == nullptr) != (v_cache == nullptr))
+    return fail(QI21_ERR_INVALID_ARG, "k_cache and v_cache must both be given or both be NULL");
+  if (B == 0 || H == 0 || L == 0) return QI21_OK;
+  QI21_TRY(check_ptr(q, "q"));
+  QI21_TRY(check_ptr(k, "k"));
+  QI21_TRY(check_ptr(v, "v"));
+  QI21_TRY(check_ptr(o, "o"));
+  QI21_TRY(check_ptr(pos, "pos"));
+  QI21_TRY(check_ptr(kv_end, "kv_end"));
+  if (k_cache != nullptr && P > 0) {
+    QI21_TRY(check_ptr(k_cache, "k_cache"));
+    QI21_TRY(check_ptr(v_cache, "v_cache"));
+  }
+  QI21_TRY(check_ptr(workspace, "workspace"));
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const WsLayout w = ws_layout(B, H, L, dt);
+  if (workspace_bytes < w.total)
+    return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float2* table = reinterpret_cast<float2*>(ws + w.table_off);
+  void* ws_k = ws + w.k_off;
+  const bool cache = k_cache != nullptr && P > 0;
+  const int64_t split = cache ? P : L;
+
+  RopePrepParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.k = k;
+  rp.v = v;
+  rp.pos = pos;
+  rp.B = B;
+  rp.H = H;
+  rp.Lk = L;
+  rp.split = split;
+  rp.k_dst0 = cache ? k_cache : ws_k;
+  rp.k_dst1 = cache ? ws_k : nullptr;
+  rp.v_dst0 = cache ? v_cache : nullptr;
+  rp.table = table;
+  rp.omega = make_omega();
+  cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
+  if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
+
+  const int64_t tokstride = (int64_t)H * kHeadDim;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.Lq = L;
+  a.q = q;
+  a.table = table;
+  a.kv_end = kv_end;
+  // keys: rows [0, split) head-major in dst0, rows [split, L) head-major in ws_k
+  a.k0 = KvSource{rp.k_dst0, split, kHeadDim, split * kHeadDim, (int64_t)H * split * kHeadDim};
+  a.k1 = KvSource{cache ? ws_k : nullptr, L - split, kHeadDim, (L - split) * kHeadDim,
+                  (int64_t)H * (L - split) * kHeadDim};
+  // values straight from v (token-major), split the same way
+  const size_t eb = elem_bytes(dt);
+  a.v0 = KvSource{v, split, tokstride, kHeadDim, L * tokstride};
+  a.v1 = KvSource{static_cast<const uint8_t*>(v) + (size_t)split * tokstride * eb, L - split, tokstride,
+                  kHeadDim, L * tokstride};
+  a.o = o;
+  a.status = status;
+  return run_attention(a, dt, st);
+}
+
+qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt, const void* q,
+                             const void* k, const void* v, const int32_t* pos_tgt, const void* k_cache,
+                             const void* v_cache, void* o, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  QI21_TRY(check_common(B, H, dt));
+  if (P < 0 || T < 0 || P > (int64_t)1 << 30 || T > (int64_t)1 << 30)
+    return fail(QI21_ERR_INVALID_ARG, "P and T must be in [0, 2^30] (P=%lld, T=%lld)", (long long)P, (long long)T);
+  if (B == 0 || H == 0 || T == 0) return QI21_OK;
+  QI21_TRY(check_ptr(q, "q"));
+  QI21_TRY(check_ptr(k, "k"));
+  QI21_TRY(check_ptr(v, "v"));
+  QI21_TRY(check_ptr(o, "o"));
+  QI21_TRY(check_ptr(pos_tgt, "pos_tgt"));
+  if (P > 0) {
+    QI21_TRY(check_ptr(k_cache, "k_cache"));
+    QI21_TRY(check_ptr(v_cache, "v_cache"));
+  }
+  QI21_TRY(check_ptr(workspace, "workspace"));
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const WsLayout w = ws_layout(B, H, T, dt);
+  if (workspace_bytes < w.total)
+    return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float2* table = reinterpret_cast<float2*>(ws + w.table_off);
+  void* ws_k = ws + w.k_off;
+
+  RopePrepParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.k = k;
+  rp.v = v;
+  rp.pos = pos_tgt;
+  rp.B = B;
+  rp.H = H;
+  rp.Lk = T;
+  rp.split = T;
+  rp.k_dst0 = ws_k;
+  rp.table = table;
+  rp.omega = make_omega();
+  cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
+  if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
+
+  const int64_t tokstride = (int64_t)H * kHeadDim;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.Lq = T;
+  a.q = q;
+  a.table = table;
+  a.kv_end = nullptr;  // the target sees every key
+  a.k0 = KvSource{k_cache, P, kHeadDim, P * kHeadDim, (int64_t)H * P * kHeadDim};
+  a.k1 = KvSource{ws_k, T, kHeadDim, T * kHeadDim, (int64_t)H * T * kHeadDim};
+  a.v0 = KvSource{v_cache, P, kHeadDim, P * kHeadDim, (int64_t)H * P * kHeadDim};
+  a.v1 = KvSource{v, T, tokstride, kHeadDim, T * tokstride};
+  a.o = o;
+  a.status = status;
+  return run_attention(a, dt, st);
+}
+
+qi21_status qi21_workspace_status(void* workspace, void* stream) {
+  if (workspace == nullptr) return fail(QI21_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WsHeader h;
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (h.status == QI21_OK) return QI21_OK;
+  const WsHeader zero = {0, 0};
+  e = cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  return fail(static_cast<qi21_status>(h.status), "device wait ran out (site 0x%x)", h.where);
+}
+
+qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream) {
+  QI21_TRY(check_ptr(workspace, "workspace"));
+  if (limit_ns < 1 || limit_ns > 2000000000LL)
+    return fail(QI21_ERR_INVALID_ARG, "limit_ns must be in [1, 2e9]");
+  cudaError_t e = launch_wait_selftest(static_cast<uint32_t*>(workspace), (uint64_t)limit_ns,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return QI21_OK;
+}
+
+void qi21_time_next_attention(void* start, void* stop) {
+  g_time_start = static_cast<cudaEvent_t>(start);
+  g_time_stop = static_cast<cudaEvent_t>(stop);
+}
+
+const char* qi21_status_string(qi21_status s) {
+  switch (s) {
+    case QI21_OK: return "QI21_OK";
+    case QI21_ERR_INVALID_ARG: return "QI21_ERR_INVALID_ARG";
+    case QI21_ERR_UNSUPPORTED: return "QI21_ERR_UNSUPPORTED";
+    case QI21_ERR_CUDA: return "QI21_ERR_CUDA";
+    case QI21_ERR_TIMEOUT: return "QI21_ERR_TIMEOUT";
+  }
+  return "QI21_ERR_UNKNOWN";
+}
+
+const char* qi21_last_error(void) { return g_last_error; }
+
+uint64_t qi21_launch_count(void) { return g_launches; }
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+// Position table builder, axial-rotation / cache pre-pass and the wait
+// self-test kernel of libqi21.
+#include <math.h>
+
+#include "qi21_device.cuh"
+#include "qi21_internal.h"
+
+namespace qi21 {
+
+// ============================================================== positions ==
+// One thread per token.  "3A - 3D Axial RoPE (16, 56, 56) & Zero-Centered
+// Grid", section 1: text advances (f, h, w) together by +1 (counting text
+// tokens only, from 0); an image freezes f and centres its row-major grid,
+// h = r - (H - H//2), w = c - (W - W//2).  Visibility bound (overview card 3C):
+// text token i sees [0, i]; an image token sees up to the end of its image.
+__global__ void positions_kernel(const __grid_constant__ PositionsParams p) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= p.L) return;
+  // last segment whose start <= i
+  int lo = 0, hi = p.n_segs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.segs[mid].start <= i) lo = mid; else hi = mid - 1;
+  }
+  const SegDev s = p.segs[lo];
+  const int32_t t = static_cast<int32_t>(i - s.start);
+  int32_t f, h, w, end;
+  if (s.kind == 0) {
+    f = h = w = s.text_base + t;
+    end = static_cast<int32_t>(i) + 1;
+  } else {
+    const int32_t r = t / s.W;
+    const int32_t c = t - r * s.W;
+    f = s.frame;
+    h = r - (s.H - s.H / 2);
+    w = c - (s.W - s.W / 2);
+    end = s.start + s.H * s.W;
+  }
+  p.pos[3 * i + 0] = f;
+  p.pos[3 * i + 1] = h;
+  p.pos[3 * i + 2] = w;
+  if (p.kv_end != nullptr) p.kv_end[i] = end;
+}
+
+cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream) {
+  if (p.L == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (p.L + threads - 1) / threads;
+  positions_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// ============================================== rotation / cache pre-pass ==
+// Per token: the 64 (cos, sin) pairs of its axial angles, computed in float64
+// and rounded once to fp32.  Pair m < 8 uses the frame axis, m < 36 the
+// height axis, the rest the width axis ("3A", section 1: bands 16/56/56).
+// Every K row is rotated once here and stored head-major (the Prefix rows go
+// straight into the KV cache); V's prefix rows are copied into the V cache.
+
+Omega make_omega() {
+  Omega o;
+  const int dims[3] = {16, 56, 56};
+  int m = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int j = 0; j < dims[a] / 2; ++j) o.w[m++] = pow(10000.0, -2.0 * j / dims[a]);
+  return o;
+}
+
+constexpr int kPrepTokens = 16;  // tokens per CTA
+constexpr int kPrepThreads = 256;
+
+template <typename T>
+struct Vec16;  // 16-byte vector of T
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+};
+
+__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, __nv_bfloat16*) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = unpack_bf16x2(w[e]);
+    const float2 r = cs[e];
+    const float y0 = fmaf(x.x, r.x, -x.y * r.y);
+    const float y1 = fmaf(x.x, r.y, x.y * r.x);
+    w[e] = pack_bf16x2(y0, y1);
+  }
+}
+__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float*) {
+  float* x = reinterpret_cast<float*>(&u);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float2 r = cs[e];
+    const float x0 = x[2 * e], x1 = x[2 * e + 1];
+    x[2 * e] = fmaf(x0, r.x, -x1 * r.y);
+    x[2 * e + 1] = fmaf(x0, r.y, x1 * r.x);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPrepThreads)
+    rope_prep_kernel(const __grid_constant__ RopePrepParams p) {
+  __shared__ float2 cs[kPrepTokens][kPairs];
+  const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kPrepTokens;
+  const int b = blockIdx.y;
+  const int ntok = static_cast<int>(p.Lk - tok0 < kPrepTokens ? p.Lk - tok0 : kPrepTokens);
+
+  for (int e = threadIdx.x; e < ntok * kPairs; e += blockDim.x) {
+    const int t = e / kPairs, m = e % kPairs;
+    const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
+    const double ang = static_cast<double>(p.pos[3 * (tok0 + t) + axis]) * p.omega.w[m];
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    const float2 v = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+    cs[t][m] = v;
+    if (p.table != nullptr && b == 0) p.table[(tok0 + t) * kPairs + m] = v;
+  }
+  __syncthreads();
+
+  constexpr int EPC = Vec16<T>::N;          // elements per 16-byte chunk
+  constexpr int CPR = kHeadDim / EPC;       // chunks per head row
+  const int H = p.H;
+  const int items = ntok * H * CPR;
+  const T* k = static_cast<const T*>(p.k);
+  const T* v = static_cast<const T*>(p.v);
+  for (int e = threadIdx.x; e < items; e += blockDim.x) {
+    const int t = e / (H * CPR);
+    const int rem = e - t * (H * CPR);
+    const int h = rem / CPR;
+    const int c = rem - h * CPR;
+    const int64_t tok = tok0 + t;
+    const int64_t src = ((static_cast<int64_t>(b) * p.Lk + tok) * H + h) * kHeadDim + c * EPC;
+    uint4 u = *reinterpret_cast<const uint4*>(k + src);
+    rotate_chunk(u, &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
+    T* dst;
+    int64_t row, rows;
+    if (tok < p.split) {
+      dst = static_cast<T*>(p.k_dst0);
+      row = tok;
+      rows = p.split;
+    } else {
+      dst = static_cast<T*>(p.k_dst1);
+      row = tok - p.split;
+      rows = p.Lk - p.split;
+    }
+    const int64_t dsti = ((static_cast<int64_t>(b) * H + h) * rows + row) * kHeadDim + c * EPC;
+    *reinterpret_cast<uint4*>(dst + dsti) = u;
+    if (p.v_dst0 != nullptr && tok < p.split) {
+      const uint4 vv = *reinterpret_cast<const uint4*>(v + src);
+      *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) + dsti) = vv;
+    }
+  }
+}
+
+cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream) {
+  if (p.Lk == 0 || p.B == 0 || p.H == 0) {
+    // the table still has to exist for zero heads/batches: nothing reads it then
+    return cudaSuccess;
+  }
+  dim3 grid(static_cast<unsigned>((p.Lk + kPrepTokens - 1) / kPrepTokens),
+            static_cast<unsigned>(p.B));
+  if (f32)
+    rope_prep_kernel<float><<<grid, kPrepThreads, 0, stream>>>(p);
+  else
+    rope_prep_kernel<__nv_bfloat16><<<grid, kPrepThreads, 0, stream>>>(p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// ============================================================ self test ==
+// One CTA waits on a barrier that no one arrives at, with a short limit; the
+// bounded wait must give up, record QI21_ERR_TIMEOUT and let the CTA exit.
+__global__ void wait_selftest_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, status, 0xFFu, limit_ns);
+  }
+  __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace qi21

@@ -1,0 +1,93 @@
+// Internal declarations shared by the host entry points and the kernels of
+// libqi21.  Not part of the public C ABI (include/qi21.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qi21 {
+
+constexpr int kHeadDim = 128;
+constexpr int kPairs = 64;           // complex pairs per head (8 + 28 + 28)
+constexpr int kBandPairs0 = 8;       // frame band: dims [0, 16)
+constexpr int kBandPairs01 = 36;     // frame + height bands: dims [0, 72)
+constexpr uint32_t kStatusTimeout = 4;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded device waits: 1 s
+
+// Status words at the start of every workspace.
+struct WsHeader {
+  uint32_t status;  // 0 = OK, else a qi21_status
+  uint32_t where;   // which wait ran out (role << 8 | barrier id)
+};
+
+// ---------------------------------------------------------------- positions
+struct SegDev {
+  int32_t kind, n, H, W, frame;
+  int32_t start;      // first token of the segment
+  int32_t text_base;  // text tokens before the segment
+};
+constexpr int kMaxSegments = 128;
+struct PositionsParams {
+  SegDev segs[kMaxSegments];
+  int32_t n_segs;
+  int64_t L;
+  int32_t* pos;
+  int32_t* kv_end;
+};
+cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream);
+
+// ------------------------------------------------- rotation / cache pre-pass
+// Angular frequency of every pair: theta^(-2j/d_axis) for its band, float64.
+struct Omega {
+  double w[kPairs];
+};
+Omega make_omega();
+
+struct RopePrepParams {
+  const void* k;       // token-major [B, Lk, H, 128]
+  const void* v;       // token-major [B, Lk, H, 128] (read only when v_dst0)
+  const int32_t* pos;  // [Lk][3]
+  int32_t B, H;
+  int64_t Lk;
+  int64_t split;   // tokens [0, split) -> dst0, [split, Lk) -> dst1
+  void* k_dst0;    // head-major [B, H, split, 128]
+  void* k_dst1;    // head-major [B, H, Lk - split, 128] (or null when split == Lk)
+  void* v_dst0;    // head-major [B, H, split, 128] copy of V, or null
+  float2* table;   // [Lk][64] (cos, sin) of every token, or null
+  Omega omega;
+};
+cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream);
+
+// --------------------------------------------------------------- attention
+// One key/value source: rows of one (batch, head) are `row` elements apart,
+// heads `head` apart, batches `batch` apart (element strides).
+struct KvSource {
+  const void* ptr;
+  int64_t n;  // rows in this source
+  int64_t row, head, batch;
+};
+
+// Attention of Lq query rows over the keys [src0 rows || src1 rows]:
+// O = softmax(rot(Q) K^T / sqrt(128) + M) V, M from kv_end (null = no mask).
+struct AttnArgs {
+  int32_t B, H;
+  int64_t Lq;
+  const void* q;          // token-major [B, Lq, H, 128] (not rotated)
+  const float2* table;    // [Lq][64] cos/sin of the query rows
+  const int32_t* kv_end;  // [Lq] or null
+  KvSource k0, k1;        // rotated keys
+  KvSource v0, v1;        // values
+  void* o;                // token-major [B, Lq, H, 128]
+  uint32_t* status;       // workspace header status word
+};
+cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);
+
+// --------------------------------------------------------------- self test
+cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+// Launch bookkeeping (thread-local counter of launches enqueued).
+void note_launch();
+
+}  // namespace qi21

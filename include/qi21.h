@@ -1,0 +1,183 @@
+/*
+ * qi21.h -- C ABI of libqi21, the sm_100a (B200) hot path of the Qwen-Image-2.1
+ * denoiser's joint attention: 3D axial RoPE, the Block-Causal mask and the
+ * Prefix KV Cache.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Head dimension is fixed at 128, split into rotary bands (16, 56, 56) for
+ *   the (frame, height, width) axes, theta = 10000, adjacent-pair rotation
+ *   ("3A - 3D Axial RoPE (16, 56, 56)", section 1; "Qwen-Image-Edit close
+ *   reading", section 7.1).  Softmax scale is 1/sqrt(128).
+ * - Activations are contiguous [B, L, H, 128] (token-major), as the joint
+ *   attention sees them after unflattening heads ("Qwen-Image-Edit close
+ *   reading", section 6 and the shape table of section 8.2).  The KV cache is
+ *   contiguous [B, H, P, 128] (head-major).
+ * - Pointers named "device" must be device memory of the current CUDA device;
+ *   every device buffer must be 16-byte aligned.  The caller owns every buffer;
+ *   the library allocates nothing and keeps no state between calls.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Calls validate their arguments on the host, enqueue kernels on `stream` and
+ *   return without synchronising.  A failed launch returns QI21_ERR_CUDA.
+ * - Errors: a non-OK status means nothing was enqueued (argument errors) or the
+ *   launch failed; qi21_last_error() returns a message for the calling thread.
+ * - Device-side waits are bounded (about one second); a wait that runs out
+ *   sets a status word in the workspace header and the kernel returns early.
+ *   qi21_workspace_status() reads and clears that word.
+ */
+#ifndef QI21_H
+#define QI21_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QI21_OK = 0,
+  QI21_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or workspace */
+  QI21_ERR_UNSUPPORTED = 2, /* valid request this build does not handle */
+  QI21_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  QI21_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out */
+} qi21_status;
+
+typedef enum {
+  QI21_BF16 = 0, /* bf16 storage, fp32 accumulation (tcgen05 tensor cores) */
+  QI21_F32 = 1   /* fp32 storage and arithmetic (CUDA cores) */
+} qi21_dtype;
+
+typedef enum { QI21_SEG_TEXT = 0, QI21_SEG_IMAGE = 1 } qi21_segment_kind;
+
+/* One segment of the joint sequence, in sequence order.  Text: `n` tokens
+ * (H, W, frame ignored).  Image: an H x W latent grid in row-major order
+ * (width fastest), all tokens sharing frame index `frame` (n ignored). */
+typedef struct {
+  int32_t kind;  /* qi21_segment_kind */
+  int32_t n;     /* text token count */
+  int32_t H, W;  /* image grid */
+  int32_t frame; /* image frame index */
+} qi21_segment;
+
+/* Bytes of the workspace header (status word); workspaces start with it. */
+#define QI21_WORKSPACE_HEADER_BYTES 256
+/* Most segments one qi21_rope_positions call accepts. */
+#define QI21_MAX_SEGMENTS 128
+
+/*
+ * qi21_rope_positions -- position table and block-causal visibility bound.
+ *
+ * Follows "3A - 3D Axial RoPE (16, 56, 56) & Zero-Centered Grid", section 1
+ * and its glossary: text tokens advance frame = height = width by +1 (the
+ * counter starts at 0 and counts text tokens only); an image keeps its frame
+ * index over the whole image and centres its grid, height running from
+ * -(H - H//2) to H//2 - 1 and width likewise.  The visibility bound follows
+ * the Block-Causal mask of the "Qwen-Image-2.1 architecture" overview (card
+ * 3C): text token i sees keys [0, i]; an image token sees every key before its
+ * image and its whole image.  Hence allowed(i, j) <=> j < kv_end[i].
+ *
+ *   segs    host array of n_segs segments (1 <= n_segs <= QI21_MAX_SEGMENTS);
+ *           text n >= 1, image H, W >= 1.
+ *   L       total tokens; must equal the sum over segments.
+ *   pos     device int32 [L][3] (frame, height, width), written.
+ *   kv_end  device int32 [L], written; may be NULL.
+ * Returns QI21_ERR_INVALID_ARG when the segments are malformed or do not add
+ * up to L.  L = 0 with n_segs = 0 is a no-op.
+ */
+qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_t L,
+                                int32_t* pos, int32_t* kv_end, void* stream);
+
+/* Workspace bytes qi21_attn_full needs for these sizes (header included). */
+size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt);
+
+/*
+ * qi21_attn_full -- the first denoising step: block-causal joint attention over
+ * the whole sequence, optionally storing the Prefix KV Cache.
+ *
+ * O = softmax(rot(Q) rot(K)^T / sqrt(128) + M) V with M[i][j] = 0 if
+ * j < kv_end[i] else -inf (overview cards 3C and 4A); key tiles that are fully
+ * masked for a query tile are skipped.  The first P tokens form the Prefix
+ * (text + reference images, before the target image); when k_cache/v_cache
+ * are given, the rotated prefix K and the prefix V are stored there for the
+ * later steps (overview card 6A: step 1 stores, steps 2..N load).
+ *
+ *   B, H, L     batch, heads, tokens (B, H >= 0; L >= 0).
+ *   P           prefix length, 0 <= P <= L.
+ *   dt          QI21_BF16 or QI21_F32; every tensor argument has this type.
+ *   q, k, v     device [B, L, H, 128], read.
+ *   pos         device int32 [L][3] from qi21_rope_positions.
+ *   kv_end      device int32 [L] from qi21_rope_positions; must be
+ *               non-decreasing with 1 <= kv_end[i] <= L (the builder's output
+ *               always is).
+ *   o           device [B, L, H, 128], written.
+ *   k_cache     device [B, H, P, 128] or NULL: rotated prefix K, written.
+ *   v_cache     device [B, H, P, 128] or NULL: prefix V, written (both or
+ *               neither must be given).
+ *   workspace   device scratch of at least qi21_attn_full_workspace_size()
+ *               bytes, 256-byte aligned; its header must be zero before the
+ *               first use (a zeroed allocation) and is kept zero by the
+ *               library unless a bounded wait runs out.
+ * Calls on one workspace must be stream-ordered.
+ */
+qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
+                           const void* q, const void* k, const void* v,
+                           const int32_t* pos, const int32_t* kv_end, void* o,
+                           void* k_cache, void* v_cache,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes qi21_attn_cached needs for these sizes (header included). */
+size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt);
+
+/*
+ * qi21_attn_cached -- a later denoising step: only the T target tokens are
+ * computed.  Their queries attend, with no mask (the target sees everything),
+ * the cached prefix keys/values followed by their own fresh keys/values:
+ * O_t = softmax(rot(Q_t) [Kc || rot(K_t)]^T / sqrt(128)) [Vc || V_t]
+ * (overview card 6A and learning goals).
+ *
+ *   B, H, P, T  batch, heads, cached prefix length (>= 0), target tokens (>= 0).
+ *   q, k, v     device [B, T, H, 128] target tensors, read.
+ *   pos_tgt     device int32 [T][3]: the target rows of the position table.
+ *   k_cache     device [B, H, P, 128] rotated prefix K from qi21_attn_full.
+ *   v_cache     device [B, H, P, 128] prefix V from qi21_attn_full.
+ *   o           device [B, T, H, 128], written.
+ *   workspace   as for qi21_attn_full, sized by qi21_attn_cached_workspace_size().
+ */
+qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                             const void* q, const void* k, const void* v,
+                             const int32_t* pos_tgt, const void* k_cache, const void* v_cache,
+                             void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the status word in the
+ * workspace header: QI21_OK, or QI21_ERR_TIMEOUT if a device wait ran out. */
+qi21_status qi21_workspace_status(void* workspace, void* stream);
+
+/* Test hook for the bounded-wait machinery: launches one CTA that waits on a
+ * shared-memory barrier nobody arrives at, with a limit of `limit_ns`
+ * nanoseconds (1..2e9).  The kernel records QI21_ERR_TIMEOUT in the workspace
+ * header and exits normally; read it with qi21_workspace_status(). */
+qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
+
+/* Profiling hook.  When `start` and `stop` are cudaEvent_t handles (passed
+ * as void*), the next attention-kernel launch made by this thread (through
+ * qi21_attn_full or qi21_attn_cached) is bracketed by cudaEventRecord(start)
+ * and cudaEventRecord(stop) on its launch stream -- the attention kernel only,
+ * not the rotation pre-pass -- after which the hook clears itself.  NULLs turn
+ * it off.  The events stay owned by the caller. */
+void qi21_time_next_attention(void* start, void* stop);
+
+const char* qi21_status_string(qi21_status s);
+
+/* Message describing the last non-OK status returned to the calling thread. */
+const char* qi21_last_error(void);
+
+/* Number of kernel launches the calling thread has enqueued through this
+ * library since it was loaded (every entry point counts its launches). */
+uint64_t qi21_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QI21_H */

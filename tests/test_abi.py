@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI that need no GPU: every symbol include/qi21.h
+declares is exported by libqi21.so, and argument validation rejects bad calls
+before anything is enqueued."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from diffusion_transformer_joint_axial_b200 import _binding as qb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qi21.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qi21_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(qb.LIB_PATH):
+        pytest.skip("libqi21.so not built")
+    return qb.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(qb.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "QI21_OK"), (1, "QI21_ERR_INVALID_ARG"), (2, "QI21_ERR_UNSUPPORTED"),
+                       (3, "QI21_ERR_CUDA"), (4, "QI21_ERR_TIMEOUT")]:
+        assert lib.qi21_status_string(code).decode() == name
+
+
+def test_workspace_sizes(lib):
+    full = lib.qi21_attn_full_workspace_size(1, 24, 4352, 256, qb.QI21_BF16)
+    # header + cos/sin table (L x 64 float2) + rotated keys (B x H x L x 128 bf16)
+    assert full >= 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
+    assert full % 256 == 0
+    cached = lib.qi21_attn_cached_workspace_size(1, 24, 256, 4096, qb.QI21_BF16)
+    assert cached >= 256 + 4096 * 64 * 8 + 24 * 4096 * 128 * 2
+    assert lib.qi21_attn_full_workspace_size(-1, 1, 1, 0, 0) == 0
+
+
+def _segs(*items):
+    arr = (qb.Segment * max(1, len(items)))()
+    for i, it in enumerate(items):
+        arr[i] = qb.Segment(*it)
+    return arr
+
+
+@pytest.mark.parametrize("segs,L", [
+    (((0, 0, 0, 0, 0),), 0),          # text with n = 0
+    (((1, 0, 0, 4, 0),), 0),          # image with H = 0
+    (((7, 3, 0, 0, 0),), 3),          # unknown kind
+    (((0, 3, 0, 0, 0),), 4),          # L does not match
+])
+def test_positions_rejects_bad_segments(lib, segs, L):
+    arr = _segs(*segs)
+    dummy = ctypes.c_void_p(16)
+    st = lib.qi21_rope_positions(arr, len(segs), L, dummy, dummy, None)
+    assert st == qb.QI21_ERR_INVALID_ARG
+    assert lib.qi21_last_error().decode()
+
+
+def test_positions_rejects_too_many_segments(lib):
+    arr = _segs(*[(0, 1, 0, 0, 0)] * 129)
+    st = lib.qi21_rope_positions(arr, 129, 129, ctypes.c_void_p(16), None, None)
+    assert st == qb.QI21_ERR_INVALID_ARG
+
+
+def test_positions_empty_is_noop(lib):
+    assert lib.qi21_rope_positions(None, 0, 0, None, None, None) == qb.QI21_OK
+
+
+def _full(lib, **kw):
+    a = dict(B=1, H=2, L=32, P=16, dt=qb.QI21_F32, q=16, k=16, v=16, pos=16, kv=16, o=16,
+             kc=None, vc=None, ws=256, wsb=1 << 30)
+    a.update(kw)
+    p = lambda x: ctypes.c_void_p(x) if x is not None else None
+    return lib.qi21_attn_full(a["B"], a["H"], a["L"], a["P"], a["dt"], p(a["q"]), p(a["k"]), p(a["v"]),
+                              p(a["pos"]), p(a["kv"]), p(a["o"]), p(a["kc"]), p(a["vc"]), p(a["ws"]),
+                              a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(P=33), qb.QI21_ERR_INVALID_ARG),            # P > L
+    (dict(P=-1), qb.QI21_ERR_INVALID_ARG),
+    (dict(B=-1), qb.QI21_ERR_INVALID_ARG),
+    (dict(dt=5), qb.QI21_ERR_UNSUPPORTED),
+    (dict(q=None), qb.QI21_ERR_INVALID_ARG),           # NULL input
+    (dict(k=24), qb.QI21_ERR_INVALID_ARG),             # misaligned
+    (dict(kc=16), qb.QI21_ERR_INVALID_ARG),            # k_cache without v_cache
+    (dict(ws=272), qb.QI21_ERR_INVALID_ARG),           # workspace not 256-aligned
+    (dict(wsb=100), qb.QI21_ERR_INVALID_ARG),          # workspace too small
+])
+def test_attn_full_rejects(lib, kw, code):
+    assert _full(lib, **kw) == code
+
+
+def test_attn_full_empty_is_noop(lib):
+    assert _full(lib, L=0, P=0, q=None, k=None, v=None, o=None, ws=None) == qb.QI21_OK
+    assert _full(lib, B=0, q=None, ws=None) == qb.QI21_OK
+    assert _full(lib, H=0, q=None, ws=None) == qb.QI21_OK
+
+
+def test_attn_cached_rejects(lib):
+    p = ctypes.c_void_p
+    ok = [p(16)] * 3
+    args = lambda P, T, kc, ws, wsb: (1, 2, P, T, qb.QI21_BF16, *ok, p(16), kc, p(16), p(16), ws, wsb, None)
+    assert lib.qi21_attn_cached(*args(-1, 4, p(16), p(256), 1 << 30)) == qb.QI21_ERR_INVALID_ARG
+    assert lib.qi21_attn_cached(*args(4, 4, None, p(256), 1 << 30)) == qb.QI21_ERR_INVALID_ARG
+    assert lib.qi21_attn_cached(*args(4, 4, p(16), p(256), 10)) == qb.QI21_ERR_INVALID_ARG
+    assert lib.qi21_attn_cached(*args(4, 0, p(16), p(256), 10)) == qb.QI21_OK  # T = 0: nothing to do
+
+
+def test_selftest_rejects_bad_limit(lib):
+    assert lib.qi21_selftest_wait_timeout(ctypes.c_void_p(256), 0, None) == qb.QI21_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_cuda(monkeypatch):
+    import torch
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
+    with pytest.raises(qb.QI21Error):
+        qb.rope_positions([{"kind": "text", "n": 4}])
