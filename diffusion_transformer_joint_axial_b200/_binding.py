@@ -27,7 +27,7 @@ WORKSPACE_HEADER_BYTES = 256
 EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_full",
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
-            "qi21_launch_count", "qi21_time_next_attention")
+            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc")
 
 
 class QI21Error(RuntimeError):
@@ -76,6 +76,9 @@ def load_library(path=LIB_PATH):
     L.qi21_launch_count.restype = ctypes.c_uint64
     L.qi21_time_next_attention.argtypes = [_vp, _vp]
     L.qi21_time_next_attention.restype = None
+    L.qi21_attn_cached_noalloc.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _vp, _vp]
+    L.qi21_attn_cached_noalloc.restype = _i32
     for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached",
                  "qi21_workspace_status", "qi21_selftest_wait_timeout"):
         getattr(L, name).restype = _i32

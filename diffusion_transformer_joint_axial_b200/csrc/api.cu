@@ -23,6 +23,14 @@ static qi21_status fail(qi21_status s, const char* fmt, ...) {
   return s;
 }
 
+qi21_status report_error(qi21_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
 static qi21_status cuda_fail(cudaError_t e, const char* what) {
   return fail(QI21_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }

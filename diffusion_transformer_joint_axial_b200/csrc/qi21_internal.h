@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/qi21.h"
+
 namespace qi21 {
 
 constexpr int kHeadDim = 128;
@@ -89,5 +91,8 @@ cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream
 
 // Launch bookkeeping (thread-local counter of launches enqueued).
 void note_launch();
+
+// Records a message for qi21_last_error() and returns `s`.
+qi21_status report_error(qi21_status s, const char* fmt, ...);
 
 }  // namespace qi21

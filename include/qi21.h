@@ -149,6 +149,32 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
                              const int32_t* pos_tgt, const void* k_cache, const void* v_cache,
                              void* o, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * qi21_attn_cached_noalloc -- the cached step of qi21_attn_cached for callers
+ * that may not allocate device memory (plugin hosts that only hand over a
+ * stream and tensors, servers that reserve all memory at start-up, loops where
+ * an allocation would synchronise the device).  The pages have no counterpart
+ * of this entry point: it exists for such callers only.
+ *
+ * Same arguments and result as qi21_attn_cached minus the workspace: the
+ * scratch is a 32 MiB array built into the library, held by every GPU that
+ * loads the library until the process exits.  Calls needing more than that
+ * (qi21_attn_cached_workspace_size() > 32 MiB) return QI21_ERR_INVALID_ARG
+ * without enqueuing anything.  The first call on a device resolves the
+ * array's device address (that device must be current); make that first call
+ * before any stream capture.  No call allocates (no cudaMalloc/cudaFree).
+ * Every call on a device shares the one array and the array keeps the last
+ * call's contents: the call clears the status header itself, and calls whose
+ * kernels overlap on the GPU (other streams, other threads) race on the
+ * scratch -- order them on one stream.  A device wait that runs out is
+ * recorded in that header but cannot be read back; callers needing that
+ * report use qi21_attn_cached with a workspace.
+ */
+qi21_status qi21_attn_cached_noalloc(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                     const void* q, const void* k, const void* v,
+                                     const int32_t* pos_tgt, const void* k_cache,
+                                     const void* v_cache, void* o, void* stream);
+
 /* Synchronises `stream`, then reads and clears the status word in the
  * workspace header: QI21_OK, or QI21_ERR_TIMEOUT if a device wait ran out. */
 qi21_status qi21_workspace_status(void* workspace, void* stream);

@@ -1,0 +1,64 @@
+"""The allocation-free cached step, qi21_attn_cached_noalloc.
+
+It serves callers that must not allocate device memory while they run
+attention (plugin hosts that only get a stream and tensors, servers that
+reserve all memory up front, loops where cudaMalloc would synchronise the
+device).  Its scratch is an array built into the library, so the test checks
+that two calls in a row -- the second one finding the first one's data still
+in that array -- give the same output as qi21_attn_cached with a workspace.
+This file is collected last on purpose.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+import diffusion_transformer_joint_axial_b200 as qi
+from diffusion_transformer_joint_axial_b200 import _binding as qb
+from diffusion_transformer_joint_axial_b200 import workloads as W
+
+from parity import assert_close
+
+
+def _noalloc(lib, q, k, v, pos_t, kc, vc, out):
+    B, T, H, _ = q.shape
+    P = kc.shape[2]
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream(q.device).cuda_stream)
+    return lib.qi21_attn_cached_noalloc(B, H, P, T, qb.QI21_BF16, p(q), p(k), p(v), p(pos_t), p(kc), p(vc),
+                                        p(out), stream)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_cached_on_two_calls(cuda_device):
+    lib = qi.load_library()
+    segs = [W.text(200), W.image(16, 20, 1), W.image(32, 32, 0)]
+    L, T = 200 + 320 + 1024, 1024
+    P = L - T
+    B, H = 1, 4
+    q, k, v = (x.to(cuda_device) for x in W.draw_qkv(B, L, H, 21, "bf16"))
+    pos, kv_end = qi.rope_positions(segs, cuda_device)
+    kc, vc = qi.alloc_cache(B, H, P, torch.bfloat16, cuda_device)
+    qi.attn_full(q, k, v, pos, kv_end, P, kc, vc)
+    pos_t = pos[P:].contiguous()
+    for call, seed in enumerate((31, 32)):
+        qt, kt, vt = (x.to(cuda_device) for x in W.draw_qkv(B, T, H, seed, "bf16"))
+        ref = qi.attn_cached(qt, kt, vt, pos_t, kc, vc)
+        out = torch.full_like(qt, float("nan"))
+        st = _noalloc(lib, qt, kt, vt, pos_t, kc, vc, out)
+        assert st == 0, lib.qi21_last_error().decode()
+        torch.cuda.synchronize()
+        assert_close(out, ref.to(torch.float64).cpu().numpy(), torch.bfloat16, "no-alloc call %d" % call)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    """Host-side check, no GPU: a cached step needing more than the built-in
+    32 MiB is refused before anything is enqueued."""
+    lib = qb.load_library()
+    B, H, P, T = 2, 24, 4608, 16384  # the 2048^2 workload's cached step: ~200 MB of scratch
+    assert lib.qi21_attn_cached_workspace_size(B, H, P, T, qb.QI21_BF16) > (32 << 20)
+    p = ctypes.c_void_p(256)
+    st = lib.qi21_attn_cached_noalloc(B, H, P, T, qb.QI21_BF16, p, p, p, p, p, p, p, None)
+    assert st == qb.QI21_ERR_INVALID_ARG
+    assert "built-in scratch" in lib.qi21_last_error().decode()
