@@ -8,9 +8,9 @@ binding: it marshals torch tensors into that ABI and nothing else.
 
 from ._binding import (QI21Error, Segment, alloc_cache, attn_cached, attn_full, cached_workspace_size,
                        full_workspace_size, launch_count, load_library, new_workspace, rope_positions,
-                       selftest_wait_timeout, time_next_attention, workspace_status, HEAD_DIM,
+                       selftest_exp2, selftest_wait_timeout, time_next_attention, workspace_status, HEAD_DIM,
                        LIB_PATH)
 
 __all__ = ["QI21Error", "Segment", "alloc_cache", "attn_cached", "attn_full", "cached_workspace_size",
            "full_workspace_size", "launch_count", "load_library", "new_workspace", "rope_positions",
-           "selftest_wait_timeout", "time_next_attention", "workspace_status", "HEAD_DIM", "LIB_PATH"]
+           "selftest_exp2", "selftest_wait_timeout", "time_next_attention", "workspace_status", "HEAD_DIM", "LIB_PATH"]

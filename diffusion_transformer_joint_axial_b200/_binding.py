@@ -27,7 +27,7 @@ WORKSPACE_HEADER_BYTES = 256
 EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_full",
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
-            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc")
+            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2")
 
 
 class QI21Error(RuntimeError):
@@ -79,6 +79,8 @@ def load_library(path=LIB_PATH):
     L.qi21_attn_cached_noalloc.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _vp, _vp]
     L.qi21_attn_cached_noalloc.restype = _i32
+    L.qi21_selftest_exp2.argtypes = [_vp, _vp, _i64, _vp]
+    L.qi21_selftest_exp2.restype = _i32
     for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached",
                  "qi21_workspace_status", "qi21_selftest_wait_timeout"):
         getattr(L, name).restype = _i32
@@ -261,3 +263,13 @@ def time_next_attention(start, stop):
             e.record()  # torch creates the event lazily on first record
     load_library().qi21_time_next_attention(ctypes.c_void_p(start.cuda_event),
                                              ctypes.c_void_p(stop.cuda_event))
+
+
+def selftest_exp2(x):
+    """The softmax's polynomial exp2 evaluated on a float32 CUDA tensor."""
+    L_ = _cuda_lib()
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        _check(L_.qi21_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(x.device)))
+    return y

@@ -15,16 +15,23 @@
 // a row's bound (the diagonal of the text block, ragged ends) are masked
 // element-wise.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue for query tile 0 (thread = row = TMEM lane)
-//   warps 4-7  softmax + epilogue for query tile 1
-//   warp  8    TMA producer (Q tiles, K/V ring of 2 stages each)
-//   warp  9    TMEM allocator and tcgen05.mma issuer
+// Warp roles (512 threads, registers rebalanced with setmaxnreg):
+//   warps 0-3   softmax for query tile 0 (thread = row = TMEM lane), 176 regs
+//   warps 4-7   softmax for query tile 1, 176 regs
+//   warps 8-11  epilogue: O / l -> bf16 -> global for both tiles, 64 regs
+//   warp  12    TMA producer (Q tiles, K/V ring of 2 stages each), 96 regs
+//   warp  13    TMEM allocator and tcgen05.mma issuer, 96 regs
+//   warps 14-15 idle, 96 regs
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the first 64 columns of its S and is the A
-// operand of the P*V MMA, so P never touches shared memory.
+// operand of the P*V MMA, so P never touches shared memory.  P is released in
+// two halves (keys 0-63, then 64-127) so the first half of P*V runs while the
+// softmax finishes the second.
 // Issue order per key tile n: PV0(n), S0(n+1), PV1(n), S1(n+1): while one
 // softmax group works the tensor core runs the other tile's MMAs.
+// Softmax arithmetic is packed (fp32x2 FMA/ADD, 3-input max); 3 of every 8
+// column pairs of unmasked tiles take exp2 from a polynomial on the FMA pipe
+// instead of the MUFU unit, which the two softmax groups otherwise saturate.
 // Online softmax uses a lazy rescale: O and l are rescaled only when a row
 // maximum grows by more than 2^8, which keeps every P <= 256.
 #include <cudaTypedefs.h>
@@ -42,10 +49,15 @@ constexpr int BN = 128;  // keys per tile
 constexpr int kStages = 2;
 constexpr int kTileBytes = BM * kHeadDim * 2;  // 32 KB: two 64-column SW128 halves
 constexpr int kHalfBytes = kTileBytes / 2;
-constexpr int kThreads = 320;
-constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
+constexpr int kThreads = 512;
+constexpr int kWarpEpi = 8;  // first epilogue warp
+constexpr int kWarpLoad = 12;
+constexpr int kWarpMma = 13;
 constexpr uint32_t kTmemCols = 512;
+// setmaxnreg budget: 128 x (176 + 176 + 64 + 96) = 65536 = 512 threads x 128.
+constexpr int kRegsSoftmax = 176;
+constexpr int kRegsEpilogue = 64;
+constexpr int kRegsOther = 96;
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bit 4),
 // A and B bf16 (bits 7, 10), N >> 3 at bit 17, M >> 4 at bit 24; bit 16 marks
@@ -58,6 +70,10 @@ constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
 // log2(e) / sqrt(128) and the lazy-rescale threshold (8 in log2 units).
 constexpr float kScaleLog2 = 0.12751743082459868f;
 constexpr float kRescaleRaw = 8.0f / kScaleLog2;
+
+// Column pairs (index j of a 64-pair row, taken mod 8) whose exp2 runs on the
+// FMA pipe: pairs 5, 6, 7 of every 8.
+constexpr uint32_t kPolyPairMask = 0xE0u;
 
 struct Params {
   CUtensorMap tm_q;
@@ -76,9 +92,10 @@ struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
+  float row_l[2][2][BM];  // [unit parity][tile][row]: softmax -> epilogue
   uint64_t q_full[2], q_rot[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_done[2], o_free[2], l_ready[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -94,15 +111,25 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   d |= (uint64_t)2 << 61;
   return d;
 }
-// K-major operand (Q or K tile): 16-element k-step kk lives in half kk/4 at
-// byte offset 32*(kk%4) of each 128-byte row; 8-row groups are 1024 B apart.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk) {
-  return sw128_desc(tile + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+// K-major operands (Q, K tiles): the 16-element k-step kk lives in half kk/4 at
+// byte offset 32*(kk%4) of each 128-byte row; 8-row groups are 1024 B apart
+// (SBO), LBO unused.  MN-major operand (V tile, rows = keys): k-step kk is 16
+// key rows = 2048 B further; the two 64-column halves are 16 KB apart (LBO).
+
+__device__ __forceinline__ void setmaxnreg_inc_softmax() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
 }
-// MN-major operand (V tile, rows = keys): k-step kk = 16 key rows = 2048 B;
-// the two 64-column halves are 16 KB apart.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk) {
-  return sw128_desc(tile + kk * 2048, kHalfBytes, 1024);
+__device__ __forceinline__ void setmaxnreg_dec_epilogue() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+}
+__device__ __forceinline__ void setmaxnreg_dec_other() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 struct Unit {
@@ -172,6 +199,50 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, int tok_maj
   }
 }
 
+// The start-address field of a descriptor is (address >> 4) in its low 14
+// bits; shared-memory addresses stay below 256 KB, so moving a descriptor by a
+// byte offset is one 64-bit add of offset >> 4 that never carries out of the
+// field.
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t qdesc, uint64_t kdesc) {
+#pragma unroll
+  for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+    const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+    mma_ss(tmem_s, qdesc + off, kdesc + off, kIdescS, kk > 0);
+  }
+}
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t vdesc, int kk0,
+                                         bool first) {
+#pragma unroll
+  for (int kk = kk0; kk < kk0 + 4; ++kk)
+    mma_ts(tmem_o, tmem_p + kk * 8, vdesc + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+           (!first || kk > 0) ? 1u : 0u);
+}
+
+// Exponentials and bf16 packing of 32 column pairs starting at pair j0 of the
+// row; accumulates the row sum into acc.  `poly` selects the mixed
+// MUFU/polynomial path (tiles without masked columns only).
+template <bool kPoly>
+__device__ __forceinline__ void exp_pack_half(const float* sv, int j0, float2 cc, float2 nmc,
+                                              float2& acc0, float2& acc1, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int c = 2 * (j0 + j);
+    const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), cc, nmc);
+    float2 e;
+    if (kPoly && ((kPolyPairMask >> ((j0 + j) & 7)) & 1u)) {
+      e = exp2_poly2(x);
+    } else {
+      e.x = ex2_approx(x.x);
+      e.y = ex2_approx(x.y);
+    }
+    if (j & 1)
+      acc1 = __fadd2_rn(acc1, e);
+    else
+      acc0 = __fadd2_rn(acc0, e);
+    pk[j] = pack_bf16x2(e.x, e.y);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -186,9 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(smem_u32(&S.q_rot[s]), BM);
       mbar_init(smem_u32(&S.q_empty[s]), 1);
       mbar_init(smem_u32(&S.s_full[s]), 1);
+      mbar_init(smem_u32(&S.p_half[s]), BM);
       mbar_init(smem_u32(&S.p_full[s]), BM);
       mbar_init(smem_u32(&S.o_done[s]), 1);
       mbar_init(smem_u32(&S.o_free[s]), BM);
+      mbar_init(smem_u32(&S.l_ready[s]), BM);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&S.k_full[s]), 1);
@@ -218,19 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
-  if (warp == kWarpLoad) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp >= kWarpLoad) {
+    setmaxnreg_dec_other();
+    if (warp == kWarpLoad) {
+      // ---------------------------------------------------------- producer
+      // The whole warp runs the loop (every value is warp-uniform, so the
+      // TMA operands stay in uniform registers); one elected lane issues.
+      const bool leader = elect_one_sync();
       uint32_t kc = 0, vc = 0, ql[2] = {0, 0};
       bool ok = true;
       for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         for (int s = 0; s < 2 && ok; ++s) {
           if (U.N[s] == 0) continue;
-          // the MMA thread releases Q_s once per unit that used it
-          ok = mbar_wait(smem_u32(&S.q_empty[s]), (ql[s] & 1u) ^ 1u, abort_flag, p.status, 0x100 | s);
+          // the MMA warp releases Q_s once per unit that used it
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_empty[s]), (ql[s] & 1u) ^ 1u,
+                                                abort_flag, p.status, 0x100 | s));
           ++ql[s];
-          if (ok) {
+          if (ok && leader) {
             const uint32_t bar = smem_u32(&S.q_full[s]);
             mbar_arrive_expect_tx(bar, kTileBytes);
             const uint32_t dst = smem_u32(S.q[s]);
@@ -243,24 +321,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const KTile t = key_tile(p, n);
           {
             const int st = kc % kStages;
-            ok = mbar_wait(smem_u32(&S.k_empty[st]), ((kc / kStages) & 1u) ^ 1u, abort_flag,
-                           p.status, 0x110 | st);
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_empty[st]), ((kc / kStages) & 1u) ^ 1u,
+                                                  abort_flag, p.status, 0x110 | st));
             if (!ok) break;
-            const uint32_t bar = smem_u32(&S.k_full[st]);
-            mbar_arrive_expect_tx(bar, kTileBytes);
-            load_kv_tile(t.src ? &p.tm_k1 : &p.tm_k0, t.src ? p.k1_tok : p.k0_tok, smem_u32(S.k[st]),
-                         bar, t.row, U.h, U.b);
+            if (leader) {
+              const uint32_t bar = smem_u32(&S.k_full[st]);
+              mbar_arrive_expect_tx(bar, kTileBytes);
+              load_kv_tile(t.src ? &p.tm_k1 : &p.tm_k0, t.src ? p.k1_tok : p.k0_tok,
+                           smem_u32(S.k[st]), bar, t.row, U.h, U.b);
+            }
             ++kc;
           }
           {
             const int st = vc % kStages;
-            ok = mbar_wait(smem_u32(&S.v_empty[st]), ((vc / kStages) & 1u) ^ 1u, abort_flag,
-                           p.status, 0x120 | st);
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.v_empty[st]), ((vc / kStages) & 1u) ^ 1u,
+                                                  abort_flag, p.status, 0x120 | st));
             if (!ok) break;
-            const uint32_t bar = smem_u32(&S.v_full[st]);
-            mbar_arrive_expect_tx(bar, kTileBytes);
-            load_kv_tile(t.src ? &p.tm_v1 : &p.tm_v0, t.src ? p.v1_tok : p.v0_tok, smem_u32(S.v[st]),
-                         bar, t.row, U.h, U.b);
+            if (leader) {
+              const uint32_t bar = smem_u32(&S.v_full[st]);
+              mbar_arrive_expect_tx(bar, kTileBytes);
+              load_kv_tile(t.src ? &p.tm_v1 : &p.tm_v0, t.src ? p.v1_tok : p.v0_tok,
+                           smem_u32(S.v[st]), bar, t.row, U.h, U.b);
+            }
             ++vc;
           }
         }
@@ -279,12 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
-    }
-  } else if (warp == kWarpMma) {
-    // -------------------------------------------------------------- MMA
-    if (lane == 0) {
-      uint32_t kc = 0, vc = 0, qv[2] = {0, 0}, pc[2] = {0, 0}, of[2] = {0, 0};
+      __syncwarp();
+    } else if (warp == kWarpMma) {
+      // -------------------------------------------------------------- MMA
+      // The whole warp runs the loop with warp-uniform values (MMA operands
+      // stay in uniform registers); one fixed elected lane issues every
+      // tcgen05.mma and tcgen05.commit, so each commit tracks all MMAs before it.
+      const bool leader = elect_one_sync();
+      const uint64_t qdesc[2] = {sw128_desc(smem_u32(S.q[0]), 16, 1024),
+                                 sw128_desc(smem_u32(S.q[1]), 16, 1024)};
+      uint32_t kc = 0, vc = 0, qv[2] = {0, 0}, ph[2] = {0, 0}, pf[2] = {0, 0}, of[2] = {0, 0};
       bool ok = true;
+      auto wait = [&](uint64_t& bar, uint32_t parity, uint32_t where) {
+        return __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar), parity, abort_flag, p.status, where));
+      };
       for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         const int N = max(U.N[0], U.N[1]);
@@ -292,90 +382,150 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // prologue: S_s(0)
         {
           const int st = kc % kStages;
-          ok = mbar_wait(smem_u32(&S.k_full[st]), (kc / kStages) & 1u, abort_flag, p.status, 0x210);
+          ok = wait(S.k_full[st], (kc / kStages) & 1u, 0x210);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kt = smem_u32(S.k[st]);
+          const uint64_t kdesc = sw128_desc(smem_u32(S.k[st]), 16, 1024);
           for (int s = 0; s < 2 && ok; ++s) {
             if (U.N[s] == 0) continue;
-            ok = mbar_wait(smem_u32(&S.q_rot[s]), qv[s] & 1u, abort_flag, p.status, 0x220 | s);
+            ok = wait(S.q_rot[s], qv[s] & 1u, 0x220 | s);
             if (!ok) break;
             ++qv[s];
             tc_fence_after();
-            const uint32_t qt = smem_u32(S.q[s]);
-            for (int kk = 0; kk < kHeadDim / 16; ++kk)
-              mma_ss(tmem + s * BN, kmajor_desc(qt, kk), kmajor_desc(kt, kk), kIdescS, kk > 0);
-            mma_commit(smem_u32(&S.s_full[s]));
-            if (U.N[s] == 1) mma_commit(smem_u32(&S.q_empty[s]));
+            if (leader) {
+              issue_s(tmem + s * BN, qdesc[s], kdesc);
+              mma_commit(smem_u32(&S.s_full[s]));
+              if (U.N[s] == 1) mma_commit(smem_u32(&S.q_empty[s]));
+            }
+            __syncwarp();
           }
           if (!ok) break;
-          mma_commit(smem_u32(&S.k_empty[st]));
+          if (leader) mma_commit(smem_u32(&S.k_empty[st]));
+          __syncwarp();
           ++kc;
         }
         for (int n = 0; n < N && ok; ++n) {
           const int vst = vc % kStages;
-          ok = mbar_wait(smem_u32(&S.v_full[vst]), (vc / kStages) & 1u, abort_flag, p.status,
-                         0x230 | vst);
+          ok = wait(S.v_full[vst], (vc / kStages) & 1u, 0x230 | vst);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vt = smem_u32(S.v[vst]);
+          const uint64_t vdesc = sw128_desc(smem_u32(S.v[vst]), kHalfBytes, 1024);
           const int kst = kc % kStages;
-          const uint32_t kt = smem_u32(S.k[kst]);
+          const uint64_t kdesc = sw128_desc(smem_u32(S.k[kst]), 16, 1024);
           bool k_ready = false;
           for (int s = 0; s < 2 && ok; ++s) {
+            const uint32_t tS = tmem + s * BN;
+            const uint32_t tO = tmem + 256 + s * kHeadDim;
             if (n < U.N[s]) {
-              ok = mbar_wait(smem_u32(&S.p_full[s]), pc[s] & 1u, abort_flag, p.status, 0x240 | s);
+              ok = wait(S.p_half[s], ph[s] & 1u, 0x240 | s);
               if (!ok) break;
-              ++pc[s];
+              ++ph[s];
               if (n == 0) {
-                ok = mbar_wait(smem_u32(&S.o_free[s]), (of[s] & 1u) ^ 1u, abort_flag, p.status,
-                               0x250 | s);
+                ok = wait(S.o_free[s], (of[s] & 1u) ^ 1u, 0x250 | s);
                 if (!ok) break;
                 ++of[s];
               }
               tc_fence_after();
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts(tmem + 256 + s * kHeadDim, tmem + s * BN + kk * 8, mnmajor_desc(vt, kk),
-                       kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
-              if (n == U.N[s] - 1) mma_commit(smem_u32(&S.o_done[s]));
+              if (leader) issue_pv(tO, tS, vdesc, 0, n == 0);
+              __syncwarp();
+              ok = wait(S.p_full[s], pf[s] & 1u, 0x270 | s);
+              if (!ok) break;
+              ++pf[s];
+              tc_fence_after();
+              if (leader) {
+                issue_pv(tO, tS, vdesc, 4, n == 0);
+                if (n == U.N[s] - 1) mma_commit(smem_u32(&S.o_done[s]));
+              }
+              __syncwarp();
             }
             if (n + 1 < U.N[s]) {
               if (!k_ready) {
-                ok = mbar_wait(smem_u32(&S.k_full[kst]), (kc / kStages) & 1u, abort_flag, p.status,
-                               0x260 | kst);
+                ok = wait(S.k_full[kst], (kc / kStages) & 1u, 0x260 | kst);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
               }
-              const uint32_t qt = smem_u32(S.q[s]);
-              for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                mma_ss(tmem + s * BN, kmajor_desc(qt, kk), kmajor_desc(kt, kk), kIdescS, kk > 0);
-              mma_commit(smem_u32(&S.s_full[s]));
-              if (n + 2 == U.N[s]) mma_commit(smem_u32(&S.q_empty[s]));
+              if (leader) {
+                issue_s(tS, qdesc[s], kdesc);
+                mma_commit(smem_u32(&S.s_full[s]));
+                if (n + 2 == U.N[s]) mma_commit(smem_u32(&S.q_empty[s]));
+              }
+              __syncwarp();
             }
           }
           if (!ok) break;
-          mma_commit(smem_u32(&S.v_empty[vst]));
-          ++vc;
-          if (k_ready) {
-            mma_commit(smem_u32(&S.k_empty[kst]));
-            ++kc;
+          if (leader) {
+            mma_commit(smem_u32(&S.v_empty[vst]));
+            if (k_ready) mma_commit(smem_u32(&S.k_empty[kst]));
           }
+          __syncwarp();
+          ++vc;
+          if (k_ready) ++kc;
         }
       }
       // Drain: every MMA issued above completes before TMEM is released.
-      mma_commit(smem_u32(&S.drain));
+      if (leader) mma_commit(smem_u32(&S.drain));
+      __syncwarp();
       mbar_wait(smem_u32(&S.drain), 0, nullptr, nullptr, 0);
+      __syncwarp();
     }
-    __syncwarp();
+  } else if (warp >= kWarpEpi) {
+    // ------------------------------------------------------------ epilogue
+    setmaxnreg_dec_epilogue();
+    const int t = threadIdx.x & 127;  // row == TMEM lane (warp % 4 picks the lane quarter)
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t cnt[2] = {0, 0};
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      const Unit U = decode_unit(p, u);
+      for (int s = 0; s < 2 && ok; ++s) {
+        if (U.N[s] == 0) continue;
+        const uint32_t par = cnt[s] & 1u;
+        ++cnt[s];
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.l_ready[s]), par, abort_flag,
+                                              p.status, 0x400 | s));
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.o_done[s]), par, abort_flag,
+                                              p.status, 0x410 | s));
+        if (!ok) break;
+        tc_fence_after();
+        const int row = U.row0 + s * BM + t;
+        const bool valid = row < p.Lq;
+        const float inv = 1.f / S.row_l[par][s][t];
+        __nv_bfloat16* dst =
+            p.o + (((size_t)U.b * p.Lq + (valid ? row : 0)) * p.H + U.h) * kHeadDim;
+        const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
+#pragma unroll 1
+        for (int c = 0; c < kHeadDim; c += 32) {
+          uint32_t orow[32];
+          tmem_ld32(tO + c, orow);
+          tmem_wait_ld();
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
+                                   __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
+              d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&S.o_free[s]));
+      }
+    }
   } else {
-    // ------------------------------------------------- softmax / epilogue
-    const int s = warp >> 2;             // query tile of this group
-    const int t = threadIdx.x & 127;     // row in the tile == TMEM lane
+    // ------------------------------------------------------------- softmax
+    setmaxnreg_inc_softmax();
+    const int s = warp >> 2;          // query tile of this group
+    const int t = threadIdx.x & 127;  // row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + s * BN;
     const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
-    uint32_t qv = 0, sf = 0, od = 0;
+    uint32_t qv = 0, sf = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
       const Unit U = decode_unit(p, u);
@@ -387,6 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_full[s]), qv & 1u, abort_flag, p.status,
                                             0x300 | s));
       if (!ok) break;
+      const uint32_t par = qv & 1u;  // unit parity of this tile's l buffer
       ++qv;
       if (valid) {
         const float4* cs = reinterpret_cast<const float4*>(p.table + (size_t)row * kPairs);
@@ -398,14 +549,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           uint4 x = *ptr;
           const float4 r01 = __ldg(cs + 2 * c);
           const float4 r23 = __ldg(cs + 2 * c + 1);
-          const float rc[4] = {r01.x, r01.z, r23.x, r23.z};
-          const float rs[4] = {r01.y, r01.w, r23.y, r23.w};
           uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xv = unpack_bf16x2(w[e]);
-            w[e] = pack_bf16x2(fmaf(xv.x, rc[e], -xv.y * rs[e]), fmaf(xv.x, rs[e], xv.y * rc[e]));
-          }
+          float2 xv = unpack_bf16x2(w[0]);
+          w[0] = pack_bf16x2(fmaf(xv.x, r01.x, -xv.y * r01.y), fmaf(xv.x, r01.y, xv.y * r01.x));
+          xv = unpack_bf16x2(w[1]);
+          w[1] = pack_bf16x2(fmaf(xv.x, r01.z, -xv.y * r01.w), fmaf(xv.x, r01.w, xv.y * r01.z));
+          xv = unpack_bf16x2(w[2]);
+          w[2] = pack_bf16x2(fmaf(xv.x, r23.x, -xv.y * r23.y), fmaf(xv.x, r23.y, xv.y * r23.x));
+          xv = unpack_bf16x2(w[3]);
+          w[3] = pack_bf16x2(fmaf(xv.x, r23.z, -xv.y * r23.w), fmaf(xv.x, r23.w, xv.y * r23.z));
           *ptr = x;
         }
       }
@@ -429,20 +581,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         float* sv = reinterpret_cast<float*>(sr);
         const KTile kt = key_tile(p, n);
         const int lim = max(0, min(kt.cnt, kv_i - kt.j0));
-        if (__any_sync(0xffffffffu, lim < BN)) {
+        const bool masked = __any_sync(0xffffffffu, lim < BN);
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c >= lim) sv[c] = -INFINITY;
         }
-        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+        float mx0 = fmax3(sv[0], sv[1], sv[2]);
+        float mx1 = fmax3(sv[3], sv[4], sv[5]);
 #pragma unroll
-        for (int c = 4; c < BN; c += 4) {
-          mx0 = fmaxf(mx0, sv[c]);
-          mx1 = fmaxf(mx1, sv[c + 1]);
-          mx2 = fmaxf(mx2, sv[c + 2]);
-          mx3 = fmaxf(mx3, sv[c + 3]);
+        for (int c = 6; c < BN - 2; c += 4) {
+          mx0 = fmax3(mx0, sv[c], sv[c + 1]);
+          mx1 = fmax3(mx1, sv[c + 2], sv[c + 3]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float mx = fmax3(mx0, mx1, fmaxf(sv[BN - 2], sv[BN - 1]));
         float alpha = 1.f;
         bool rescale = false;
         if (n == 0) {
@@ -452,19 +604,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           m = mx;
           rescale = true;
         }
-        const float mc = m * kScaleLog2;
-        float l0 = 0.f, l1 = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(fmaf(sv[c], kScaleLog2, -mc));
-          const float p1 = ex2_approx(fmaf(sv[c + 1], kScaleLog2, -mc));
-          l0 += p0;
-          l1 += p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        const float2 cc = make_float2(kScaleLog2, kScaleLog2);
+        const float2 nmc = make_float2(-m * kScaleLog2, -m * kScaleLog2);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint32_t pk[32];
+        // ---- first half of P (keys 0-63)
+        if (masked)
+          exp_pack_half<false>(sv, 0, cc, nmc, acc0, acc1, pk);
+        else
+          exp_pack_half<true>(sv, 0, cc, nmc, acc0, acc1, pk);
+        tmem_st32(tS + 0, pk);
         if (__any_sync(0xffffffffu, rescale)) {
           // O holds PV(n-1): it is complete, since S(n) was committed after it.
 #pragma unroll 1
@@ -477,40 +626,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tmem_st32(tO + c, orow);
           }
         }
-        l = l * alpha + (l0 + l1);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&S.p_half[s]));
+        // ---- second half of P (keys 64-127)
+        if (masked)
+          exp_pack_half<false>(sv, 32, cc, nmc, acc0, acc1, pk);
+        else
+          exp_pack_half<true>(sv, 32, cc, nmc, acc0, acc1, pk);
+        tmem_st32(tS + 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&S.p_full[s]));
+        const float2 acc = __fadd2_rn(acc0, acc1);
+        l = l * alpha + (acc.x + acc.y);
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16 -> global
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.o_done[s]), od & 1u, abort_flag, p.status,
-                                            0x320 | s));
-      if (!ok) break;
-      ++od;
-      tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst =
-          p.o + (((size_t)U.b * p.Lq + (valid ? row : 0)) * p.H + U.h) * kHeadDim;
-#pragma unroll 1
-      for (int c = 0; c < kHeadDim; c += 32) {
-        uint32_t orow[32];
-        tmem_ld32(tO + c, orow);
-        tmem_wait_ld();
-        if (valid) {
-          uint32_t pkd[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pkd[e] = pack_bf16x2(__uint_as_float(orow[2 * e]) * inv,
-                                 __uint_as_float(orow[2 * e + 1]) * inv);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&S.o_free[s]));
+      S.row_l[par][s][t] = l;
+      mbar_arrive(smem_u32(&S.l_ready[s]));
     }
   }
 

@@ -88,6 +88,7 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
 
 // --------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 // Launch bookkeeping (thread-local counter of launches enqueued).
 void note_launch();

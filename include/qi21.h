@@ -185,6 +185,12 @@ qi21_status qi21_workspace_status(void* workspace, void* stream);
  * header and exits normally; read it with qi21_workspace_status(). */
 qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
 
+/* Test hook for the polynomial exp2 that the bf16 softmax evaluates on the
+ * FMA pipe for part of its columns (range reduction to [-1/2, 1/2] plus a
+ * cubic minimax fit, relative error below 1e-4 for x in [-125, 128)).
+ * Writes y[i] = 2^x[i] for n device floats (x clamped below at -125). */
+qi21_status qi21_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
 /* Profiling hook.  When `start` and `stop` are cudaEvent_t handles (passed
  * as void*), the next attention-kernel launch made by this thread (through
  * qi21_attn_full or qi21_attn_cached) is bracketed by cudaEventRecord(start)
