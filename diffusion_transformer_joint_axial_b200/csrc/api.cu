@@ -199,6 +199,7 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
   rp.k_dst1 = cache ? ws_k : nullptr;
   rp.v_dst0 = cache ? v_cache : nullptr;
   rp.table = table;
+  rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
@@ -206,6 +207,7 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
   const int64_t tokstride = (int64_t)H * kHeadDim;
   AttnArgs a;
   memset(&a, 0, sizeof(a));
+  a.unit_counter = rp.unit_counter;
   a.B = B;
   a.H = H;
   a.Lq = L;
@@ -266,6 +268,7 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
   rp.split = T;
   rp.k_dst0 = ws_k;
   rp.table = table;
+  rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
@@ -273,6 +276,7 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
   const int64_t tokstride = (int64_t)H * kHeadDim;
   AttnArgs a;
   memset(&a, 0, sizeof(a));
+  a.unit_counter = rp.unit_counter;
   a.B = B;
   a.H = H;
   a.Lq = T;

@@ -7,8 +7,9 @@
 // cache or the per-step pre-pass); M is the block-causal mask given by
 // kv_end (allowed(i, j) <=> j < kv_end[i]) or no mask at all.
 //
-// Work unit: one (batch, head) and a pair of 128-row query tiles.  A CTA
-// (one per SM, persistent) walks its units in order of decreasing cost.
+// Work unit: one (batch, head) and a pair of 128-row query tiles.  CTAs (one
+// per SM, persistent) take units from a global counter in order of decreasing
+// cost (longest-processing-time-first, decided at run time).
 // For each query tile only the key tiles that start below the tile's largest
 // kv_end are visited: every visibility bound is a prefix of the keys, so
 // fully masked tiles are skipped and never loaded; only tiles that straddle
@@ -19,9 +20,10 @@
 //   warps 0-3   softmax for query tile 0 (thread = row = TMEM lane), 176 regs
 //   warps 4-7   softmax for query tile 1, 176 regs
 //   warps 8-11  epilogue: O / l -> bf16 -> global for both tiles, 64 regs
-//   warp  12    TMA producer (Q tiles, K/V ring of 2 stages each), 96 regs
+//   warp  12    TMA producer of Q tiles and the K ring (2 stages), 96 regs
 //   warp  13    TMEM allocator and tcgen05.mma issuer, 96 regs
-//   warps 14-15 idle, 96 regs
+//   warp  14    TMA producer of the V ring (2 stages), 96 regs
+//   warp  15    idle, 96 regs
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the first 64 columns of its S and is the A
 // operand of the P*V MMA, so P never touches shared memory.  P is released in
@@ -29,9 +31,9 @@
 // softmax finishes the second.
 // Issue order per key tile n: PV0(n), S0(n+1), PV1(n), S1(n+1): while one
 // softmax group works the tensor core runs the other tile's MMAs.
-// Softmax arithmetic is packed (fp32x2 FMA/ADD, 3-input max); 3 of every 8
-// column pairs of unmasked tiles take exp2 from a polynomial on the FMA pipe
-// instead of the MUFU unit, which the two softmax groups otherwise saturate.
+// The softmax keeps its dependency chains short (eight partial row sums, an
+// eight-chain row max): on B200 a lone softmax warp per SMSP is bound by
+// instruction latency more than by the MUFU exp2 rate.
 // Online softmax uses a lazy rescale: O and l are rescaled only when a row
 // maximum grows by more than 2^8, which keeps every P <= 256.
 #include <cudaTypedefs.h>
@@ -51,8 +53,9 @@ constexpr int kTileBytes = BM * kHeadDim * 2;  // 32 KB: two 64-column SW128 hal
 constexpr int kHalfBytes = kTileBytes / 2;
 constexpr int kThreads = 512;
 constexpr int kWarpEpi = 8;  // first epilogue warp
-constexpr int kWarpLoad = 12;
+constexpr int kWarpLoad = 12;   // Q and K tiles
 constexpr int kWarpMma = 13;
+constexpr int kWarpLoadV = 14;  // V tiles
 constexpr uint32_t kTmemCols = 512;
 // setmaxnreg budget: 128 x (176 + 176 + 64 + 96) = 65536 = 512 threads x 128.
 constexpr int kRegsSoftmax = 176;
@@ -71,9 +74,11 @@ constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
 constexpr float kScaleLog2 = 0.12751743082459868f;
 constexpr float kRescaleRaw = 8.0f / kScaleLog2;
 
-// Column pairs (index j of a 64-pair row, taken mod 8) whose exp2 runs on the
-// FMA pipe: pairs 5, 6, 7 of every 8.
-constexpr uint32_t kPolyPairMask = 0xE0u;
+// Column pairs (index j of a 64-pair row, taken mod 8) whose exp2 would run on
+// the FMA pipe instead of MUFU.  Measured on B200: a softmax warp is bound by
+// instruction latency rather than by MUFU, and the polynomial's FMA work slows
+// the warps sharing its SMSP, so no pair takes the polynomial path.
+constexpr uint32_t kPolyPairMask = 0x00u;
 
 struct Params {
   CUtensorMap tm_q;
@@ -86,16 +91,23 @@ struct Params {
   const int32_t* kv_end;
   __nv_bfloat16* o;
   uint32_t* status;
+  uint32_t* unit_counter;  // zeroed by the pre-pass kernel before this launch
 };
+
+constexpr int kSchedSlots = 4;
+// Threads that read every scheduled unit: warps 0-14 (warp 15 idles).
+constexpr uint32_t kSchedReaders = 15 * 32;
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   float row_l[2][2][BM];  // [unit parity][tile][row]: softmax -> epilogue
+  int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
   uint64_t q_full[2], q_rot[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_half[2], p_full[2], o_done[2], o_free[2], l_ready[2];
+  uint64_t sched_full[kSchedSlots], sched_empty[kSchedSlots];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -219,28 +231,61 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint6
 }
 
 // Exponentials and bf16 packing of 32 column pairs starting at pair j0 of the
-// row; accumulates the row sum into acc.  `poly` selects the mixed
-// MUFU/polynomial path (tiles without masked columns only).
+// row; accumulates the row sum into eight independent partial sums (the adds
+// have a long latency: a single chain would serialise the loop).  kPoly
+// selects the mixed MUFU/polynomial path (tiles without masked columns only).
 template <bool kPoly>
-__device__ __forceinline__ void exp_pack_half(const float* sv, int j0, float2 cc, float2 nmc,
-                                              float2& acc0, float2& acc1, uint32_t (&pk)[32]) {
+__device__ __forceinline__ void exp_pack_half(const float* sv, int j0, float mc, float (&acc)[8],
+                                              uint32_t (&pk)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const int c = 2 * (j0 + j);
-    const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), cc, nmc);
-    float2 e;
+    const float x0 = fmaf(sv[c], kScaleLog2, -mc);
+    const float x1 = fmaf(sv[c + 1], kScaleLog2, -mc);
+    float e0, e1;
     if (kPoly && ((kPolyPairMask >> ((j0 + j) & 7)) & 1u)) {
-      e = exp2_poly2(x);
+      const float2 e = exp2_poly2(make_float2(x0, x1));
+      e0 = e.x;
+      e1 = e.y;
     } else {
-      e.x = ex2_approx(x.x);
-      e.y = ex2_approx(x.y);
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
     }
-    if (j & 1)
-      acc1 = __fadd2_rn(acc1, e);
-    else
-      acc0 = __fadd2_rn(acc0, e);
-    pk[j] = pack_bf16x2(e.x, e.y);
+    acc[(2 * j) & 7] += e0;
+    acc[(2 * j + 1) & 7] += e1;
+    pk[j] = pack_bf16x2(e0, e1);
   }
+}
+
+// Dynamic schedule: the K-producer warp takes the next unit from a global
+// counter (units are numbered in decreasing-cost order) and publishes it in a
+// shared-memory ring; every role reads the same sequence through next_unit().
+__device__ __forceinline__ void publish_unit(Smem& S, const Params& p, uint32_t sc, bool leader,
+                                             volatile int* abort, bool& ok) {
+  const int slot = sc % kSchedSlots;
+  ok = ok && __all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&S.sched_empty[slot]), ((sc / kSchedSlots) & 1u) ^ 1u,
+                                  abort, p.status, 0x500));
+  if (ok && leader) {
+    const uint32_t u = atomicAdd(p.unit_counter, 1u);
+    S.sched_unit[slot] = u < (uint32_t)p.num_units ? (int32_t)u : -1;
+    mbar_arrive(smem_u32(&S.sched_full[slot]));
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ int next_unit(Smem& S, const Params& p, uint32_t& sc, volatile int* abort,
+                                         bool& ok) {
+  const int slot = sc % kSchedSlots;
+  ok = ok && __all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&S.sched_full[slot]), (sc / kSchedSlots) & 1u, abort,
+                                  p.status, 0x510));
+  int u = -1;
+  if (ok) {
+    u = *reinterpret_cast<volatile int32_t*>(&S.sched_unit[slot]);
+    mbar_arrive(smem_u32(&S.sched_empty[slot]));
+  }
+  ++sc;
+  return ok ? u : -1;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
@@ -269,6 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(smem_u32(&S.v_full[s]), 1);
       mbar_init(smem_u32(&S.v_empty[s]), 1);
     }
+    for (int s = 0; s < kSchedSlots; ++s) {
+      mbar_init(smem_u32(&S.sched_full[s]), 1);
+      mbar_init(smem_u32(&S.sched_empty[s]), kSchedReaders);
+    }
     mbar_init(smem_u32(&S.drain), 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -293,16 +342,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (warp >= kWarpLoad) {
     setmaxnreg_dec_other();
-    if (warp == kWarpLoad) {
-      // ---------------------------------------------------------- producer
+    if (warp == kWarpLoad || warp == kWarpLoadV) {
+      // --------------------------------------------------------- producers
+      // Warp 12 loads Q and K, warp 14 loads V, so a wait for a free V stage
+      // never holds back the next K tile (and the other way round).
+      const bool do_qk = warp == kWarpLoad;
+      uint32_t sc = 0;
       // The whole warp runs the loop (every value is warp-uniform, so the
       // TMA operands stay in uniform registers); one elected lane issues.
       const bool leader = elect_one_sync();
       uint32_t kc = 0, vc = 0, ql[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      while (ok) {
+        if (do_qk) publish_unit(S, p, sc, leader, abort_flag, ok);
+        const int u = next_unit(S, p, sc, abort_flag, ok);
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
-        for (int s = 0; s < 2 && ok; ++s) {
+        for (int s = 0; s < 2 && ok && do_qk; ++s) {
           if (U.N[s] == 0) continue;
           // the MMA warp releases Q_s once per unit that used it
           ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_empty[s]), (ql[s] & 1u) ^ 1u,
@@ -319,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int N = max(U.N[0], U.N[1]);
         for (int n = 0; n < N && ok; ++n) {
           const KTile t = key_tile(p, n);
-          {
+          if (do_qk) {
             const int st = kc % kStages;
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_empty[st]), ((kc / kStages) & 1u) ^ 1u,
                                                   abort_flag, p.status, 0x110 | st));
@@ -331,8 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                            smem_u32(S.k[st]), bar, t.row, U.h, U.b);
             }
             ++kc;
-          }
-          {
+          } else {
             const int st = vc % kStages;
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.v_empty[st]), ((vc / kStages) & 1u) ^ 1u,
                                                   abort_flag, p.status, 0x120 | st));
@@ -375,7 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       auto wait = [&](uint64_t& bar, uint32_t parity, uint32_t where) {
         return __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar), parity, abort_flag, p.status, where));
       };
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      uint32_t sc = 0;
+      while (ok) {
+        const int u = next_unit(S, p, sc, abort_flag, ok);
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
         const int N = max(U.N[0], U.N[1]);
         if (N == 0) continue;
@@ -474,9 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     setmaxnreg_dec_epilogue();
     const int t = threadIdx.x & 127;  // row == TMEM lane (warp % 4 picks the lane quarter)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t cnt[2] = {0, 0};
+    uint32_t cnt[2] = {0, 0}, sc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    while (ok) {
+      const int u = next_unit(S, p, sc, abort_flag, ok);
+      if (u < 0) break;
       const Unit U = decode_unit(p, u);
       for (int s = 0; s < 2 && ok; ++s) {
         if (U.N[s] == 0) continue;
@@ -525,9 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + s * BN;
     const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
-    uint32_t qv = 0, sf = 0;
+    uint32_t qv = 0, sf = 0, sc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    while (ok) {
+      const int u = next_unit(S, p, sc, abort_flag, ok);
+      if (u < 0) break;
       const Unit U = decode_unit(p, u);
       const int Ns = U.N[s];
       if (Ns == 0) continue;
@@ -587,14 +649,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < BN; ++c)
             if (c >= lim) sv[c] = -INFINITY;
         }
-        float mx0 = fmax3(sv[0], sv[1], sv[2]);
-        float mx1 = fmax3(sv[3], sv[4], sv[5]);
+        // row max: eight independent chains, then a tree
+        float mxc[8];
 #pragma unroll
-        for (int c = 6; c < BN - 2; c += 4) {
-          mx0 = fmax3(mx0, sv[c], sv[c + 1]);
-          mx1 = fmax3(mx1, sv[c + 2], sv[c + 3]);
+        for (int i = 0; i < 8; ++i) mxc[i] = fmaxf(sv[i], sv[i + 8]);
+#pragma unroll
+        for (int c = 16; c < BN; c += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mxc[i] = fmax3(mxc[i], sv[c + i], sv[c + i + 8]);
         }
-        const float mx = fmax3(mx0, mx1, fmaxf(sv[BN - 2], sv[BN - 1]));
+        const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]),
+                               fmaxf(fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7])));
         float alpha = 1.f;
         bool rescale = false;
         if (n == 0) {
@@ -604,15 +669,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           m = mx;
           rescale = true;
         }
-        const float2 cc = make_float2(kScaleLog2, kScaleLog2);
-        const float2 nmc = make_float2(-m * kScaleLog2, -m * kScaleLog2);
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        const float mc = m * kScaleLog2;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         uint32_t pk[32];
         // ---- first half of P (keys 0-63)
-        if (masked)
-          exp_pack_half<false>(sv, 0, cc, nmc, acc0, acc1, pk);
+        if (masked || kPolyPairMask == 0u)
+          exp_pack_half<false>(sv, 0, mc, acc, pk);
         else
-          exp_pack_half<true>(sv, 0, cc, nmc, acc0, acc1, pk);
+          exp_pack_half<true>(sv, 0, mc, acc, pk);
         tmem_st32(tS + 0, pk);
         if (__any_sync(0xffffffffu, rescale)) {
           // O holds PV(n-1): it is complete, since S(n) was committed after it.
@@ -630,16 +694,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tc_fence_before();
         mbar_arrive(smem_u32(&S.p_half[s]));
         // ---- second half of P (keys 64-127)
-        if (masked)
-          exp_pack_half<false>(sv, 32, cc, nmc, acc0, acc1, pk);
+        if (masked || kPolyPairMask == 0u)
+          exp_pack_half<false>(sv, 32, mc, acc, pk);
         else
-          exp_pack_half<true>(sv, 32, cc, nmc, acc0, acc1, pk);
+          exp_pack_half<true>(sv, 32, mc, acc, pk);
         tmem_st32(tS + 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&S.p_full[s]));
-        const float2 acc = __fadd2_rn(acc0, acc1);
-        l = l * alpha + (acc.x + acc.y);
+        l = l * alpha + (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
       }
       if (!ok) break;
       S.row_l[par][s][t] = l;
@@ -723,6 +786,7 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.kv_end = a.kv_end;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.status = a.status;
+  p.unit_counter = a.unit_counter;
   const size_t smem = sizeof(tc::Smem) + 1024;
   cudaError_t err =
       cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

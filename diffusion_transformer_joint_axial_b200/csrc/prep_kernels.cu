@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(kPrepThreads)
   __shared__ float2 cs[kPrepTokens][kPairs];
   const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kPrepTokens;
   const int b = blockIdx.y;
+  if (p.unit_counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+    *p.unit_counter = 0u;
   const int ntok = static_cast<int>(p.Lk - tok0 < kPrepTokens ? p.Lk - tok0 : kPrepTokens);
 
   for (int e = threadIdx.x; e < ntok * kPairs; e += blockDim.x) {

@@ -55,6 +55,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps (up to `ns` nanoseconds) instead of spinning, so waiting warps do not
+// take issue slots from the warps sharing their SMSP.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up
 // after `limit_ns` nanoseconds, or when *abort becomes non-zero (another role
 // gave up; `abort` may be null to skip that check); on running out of time it
@@ -65,16 +80,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  uint32_t iter = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++iter & 63u) == 0u) {
-      if (abort != nullptr && *abort) return false;
-      if (global_ns() - t0 > limit_ns) {
-        if (abort != nullptr) *abort = 1;
-        record_status(status, kStatusTimeout, where);
-        return false;
-      }
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (global_ns() - t0 > limit_ns) {
+      if (abort != nullptr) *abort = 1;
+      record_status(status, kStatusTimeout, where);
+      return false;
     }
   }
 }

@@ -19,8 +19,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded device waits: 1 s
 
 // Status words at the start of every workspace.
 struct WsHeader {
-  uint32_t status;  // 0 = OK, else a qi21_status
-  uint32_t where;   // which wait ran out (role << 8 | barrier id)
+  uint32_t status;        // 0 = OK, else a qi21_status
+  uint32_t where;         // which wait ran out (role << 8 | barrier id)
+  uint32_t unit_counter;  // next work unit of the attention kernel's dynamic schedule
 };
 
 // ---------------------------------------------------------------- positions
@@ -57,6 +58,7 @@ struct RopePrepParams {
   void* k_dst1;    // head-major [B, H, Lk - split, 128] (or null when split == Lk)
   void* v_dst0;    // head-major [B, H, split, 128] copy of V, or null
   float2* table;   // [Lk][64] (cos, sin) of every token, or null
+  uint32_t* unit_counter;  // zeroed here for the attention launch that follows, or null
   Omega omega;
 };
 cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream);
@@ -82,6 +84,7 @@ struct AttnArgs {
   KvSource v0, v1;        // values
   void* o;                // token-major [B, Lq, H, 128]
   uint32_t* status;       // workspace header status word
+  uint32_t* unit_counter; // workspace header: dynamic-schedule counter (zeroed by the pre-pass)
 };
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);
