@@ -67,8 +67,9 @@ Omega make_omega() {
   return o;
 }
 
-constexpr int kPrepTokens = 16;  // tokens per CTA
+constexpr int kPrepTokens = 4;  // tokens per CTA: one (token, pair) angle per thread
 constexpr int kPrepThreads = 256;
+constexpr int kPrepUnroll = 4;  // 16-byte loads each thread keeps in flight
 
 template <typename T>
 struct Vec16;  // 16-byte vector of T
@@ -103,6 +104,14 @@ __device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float*)
   }
 }
 
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kPrepThreads)
     rope_prep_kernel(const __grid_constant__ RopePrepParams p) {
@@ -113,49 +122,67 @@ __global__ void __launch_bounds__(kPrepThreads)
     *p.unit_counter = 0u;
   const int ntok = static_cast<int>(p.Lk - tok0 < kPrepTokens ? p.Lk - tok0 : kPrepTokens);
 
-  for (int e = threadIdx.x; e < ntok * kPairs; e += blockDim.x) {
-    const int t = e / kPairs, m = e % kPairs;
-    const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
-    const double ang = static_cast<double>(p.pos[3 * (tok0 + t) + axis]) * p.omega.w[m];
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    const float2 v = make_float2(static_cast<float>(cd), static_cast<float>(sd));
-    cs[t][m] = v;
-    if (p.table != nullptr && b == 0) p.table[(tok0 + t) * kPairs + m] = v;
+  {
+    const int t = threadIdx.x / kPairs, m = threadIdx.x % kPairs;
+    if (t < ntok) {
+      const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
+      const double ang = static_cast<double>(p.pos[3 * (tok0 + t) + axis]) * p.omega.w[m];
+      double sd, cd;
+      sincos(ang, &sd, &cd);
+      const float2 v = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+      cs[t][m] = v;
+      if (p.table != nullptr && b == 0) p.table[(tok0 + t) * kPairs + m] = v;
+    }
   }
   __syncthreads();
 
-  constexpr int EPC = Vec16<T>::N;          // elements per 16-byte chunk
-  constexpr int CPR = kHeadDim / EPC;       // chunks per head row
+  constexpr int EPC = Vec16<T>::N;     // elements per 16-byte chunk
+  constexpr int CPR = kHeadDim / EPC;  // chunks per head row
   const int H = p.H;
   const int items = ntok * H * CPR;
-  const T* k = static_cast<const T*>(p.k);
-  const T* v = static_cast<const T*>(p.v);
-  for (int e = threadIdx.x; e < items; e += blockDim.x) {
-    const int t = e / (H * CPR);
-    const int rem = e - t * (H * CPR);
-    const int h = rem / CPR;
-    const int c = rem - h * CPR;
-    const int64_t tok = tok0 + t;
-    const int64_t src = ((static_cast<int64_t>(b) * p.Lk + tok) * H + h) * kHeadDim + c * EPC;
-    uint4 u = *reinterpret_cast<const uint4*>(k + src);
-    rotate_chunk(u, &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
-    T* dst;
-    int64_t row, rows;
-    if (tok < p.split) {
-      dst = static_cast<T*>(p.k_dst0);
-      row = tok;
-      rows = p.split;
-    } else {
-      dst = static_cast<T*>(p.k_dst1);
-      row = tok - p.split;
-      rows = p.Lk - p.split;
+  const T* __restrict__ k = static_cast<const T*>(p.k);
+  const T* __restrict__ v = static_cast<const T*>(p.v);
+  for (int e0 = threadIdx.x; e0 < items; e0 += kPrepUnroll * kPrepThreads) {
+    uint4 ku[kPrepUnroll], vu[kPrepUnroll];
+    int64_t src[kPrepUnroll];
+#pragma unroll
+    for (int i = 0; i < kPrepUnroll; ++i) {
+      const int e = e0 + i * kPrepThreads;
+      if (e < items) {
+        const int t = e / (H * CPR);
+        const int rem = e - t * (H * CPR);
+        const int h = rem / CPR;
+        const int c = rem - h * CPR;
+        src[i] = ((static_cast<int64_t>(b) * p.Lk + tok0 + t) * H + h) * kHeadDim + c * EPC;
+        ku[i] = ld_stream(k + src[i]);
+        if (p.v_dst0 != nullptr && tok0 + t < p.split) vu[i] = ld_stream(v + src[i]);
+      }
     }
-    const int64_t dsti = ((static_cast<int64_t>(b) * H + h) * rows + row) * kHeadDim + c * EPC;
-    *reinterpret_cast<uint4*>(dst + dsti) = u;
-    if (p.v_dst0 != nullptr && tok < p.split) {
-      const uint4 vv = *reinterpret_cast<const uint4*>(v + src);
-      *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) + dsti) = vv;
+#pragma unroll
+    for (int i = 0; i < kPrepUnroll; ++i) {
+      const int e = e0 + i * kPrepThreads;
+      if (e >= items) continue;
+      const int t = e / (H * CPR);
+      const int rem = e - t * (H * CPR);
+      const int h = rem / CPR;
+      const int c = rem - h * CPR;
+      const int64_t tok = tok0 + t;
+      rotate_chunk(ku[i], &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
+      T* dst;
+      int64_t row, rows;
+      if (tok < p.split) {
+        dst = static_cast<T*>(p.k_dst0);
+        row = tok;
+        rows = p.split;
+      } else {
+        dst = static_cast<T*>(p.k_dst1);
+        row = tok - p.split;
+        rows = p.Lk - p.split;
+      }
+      const int64_t dsti = ((static_cast<int64_t>(b) * H + h) * rows + row) * kHeadDim + c * EPC;
+      *reinterpret_cast<uint4*>(dst + dsti) = ku[i];
+      if (p.v_dst0 != nullptr && tok < p.split)
+        *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) + dsti) = vu[i];
     }
   }
 }
