@@ -16,6 +16,7 @@ Prints one JSON line on rank 0.
 """
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -33,6 +34,21 @@ from diffusion_transformer_joint_axial_b200 import workloads as W  # noqa: E402
 
 METRIC = "joint-attn TFLOP/s (full step & prefix-cached step), % of B200 BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) per attention launch, from the ncu capture summarised in
+# profiles/attn_tc_t2i.md (mean of the full-step and cached-step launches).  Valid only
+# for the kernel source it was taken on: a different attn_tc.cu reports null.
+NCU_TRAFFIC = {"attn_tc_source_sha256": "5401ac83cd7c399a",
+               "bytes_per_launch": {"t2i": (152.9e6 + 135.7e6) / 2}}
+
+
+def ncu_traffic(name):
+    src = os.path.join(ROOT, "diffusion_transformer_joint_axial_b200", "csrc", "attn_tc.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    if digest != NCU_TRAFFIC["attn_tc_source_sha256"]:
+        return None
+    return NCU_TRAFFIC["bytes_per_launch"].get(name)
 
 
 # ------------------------------------------------------------------ helpers --
@@ -330,7 +346,7 @@ def run_ours(args, world, rank, local):
         "cached_step": {"tflops": cached_tf, "frac_of_peak": cached_tf / peak,
                         "ms": cached_ms / args.steps},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": ncu_traffic(name), "traffic_unit": "bytes/launch",
                      "kernel": "qi21::tc::attn_tc_kernel (full + cached launches)",
                      "peak_kind": "%s bf16 dense burst (cuBLAS), MEASURED_PEAKS.json" % kind},
         "cpu_baseline": cpu,
