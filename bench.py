@@ -4,7 +4,10 @@ One step = one pass of the whole path over one batch of synthetic input:
 position table -> full block-causal step (axial RoPE, tile-skipping mask,
 Prefix KV cache store) -> one prefix-cached target-only step.  The metric is
 algorithmic TFLOP/s: 4 * 128 * (allowed query/key pairs) per (batch, head),
-masked tiles and elements excluded.
+masked tiles and elements excluded.  For the max-reference workload the line
+also carries ``loop``: the 8-step denoising loop of one layer (1 full + 7
+cached steps on fresh target inputs) timed as eager calls and as one CUDA
+graph replay.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload t2i]
     python bench.py --impl reference ...   # the float64 CPU oracle, timed
@@ -217,6 +220,45 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm --
 
+def pct(xs, q):
+    return float(np.percentile(np.asarray(xs, dtype=np.float64), q))
+
+
+def time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops):
+    """The workload's denoising loop for one layer: step 1 full (cache store)
+    and steps 2..N cached on fresh target inputs, timed eagerly (one library
+    call per step) and as one CUDA-graph replay; L2 flushed before each."""
+    n = 1 + cfg["cached_steps"]
+    loop = qi.DenoiseLoop(cfg["segments"], cfg["B"], cfg["H"], n, torch.bfloat16, dev)
+    loop.load(*W.full_inputs(name), [W.cached_inputs(name, s) for s in range(2, n + 1)])
+    loop.capture()
+    stream = torch.cuda.current_stream(dev)
+    reps = max(3, min(args.steps, 10))
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    times = {}
+    for mode, fn in (("eager", loop.run), ("graph", loop.replay)):
+        for _ in range(2):
+            fn()
+        ev = [(mk(), mk()) for _ in range(reps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        times[mode] = [a.elapsed_time(b) for a, b in ev]
+    loop.check()
+    flops = full_flops + (n - 1) * cached_flops
+    g = pct(times["graph"], 50)
+    out = {"steps": n, "calls": "1 full + %d cached" % (n - 1), "reps": reps,
+           "graph_ms_median": g, "graph_ms_p95": pct(times["graph"], 95),
+           "eager_ms_median": pct(times["eager"], 50), "eager_ms_p95": pct(times["eager"], 95),
+           "tflops_graph": flops / (g * 1e-3) / 1e12}
+    del loop
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     import diffusion_transformer_joint_axial_b200 as qi
     dev = torch.device("cuda", local)
@@ -285,9 +327,15 @@ def run_ours(args, world, rank, local):
     launches = qi.launch_count() - n0
     clk = clocks.stop() if clocks else None
     step_ms = sum(e[4].elapsed_time(e[5]) for e in evs)
-    full_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    cached_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    full_each = [e[0].elapsed_time(e[1]) for e in evs]
+    cached_each = [e[2].elapsed_time(e[3]) for e in evs]
+    full_ms, cached_ms = sum(full_each), sum(cached_each)
     assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
+
+    # ---- the denoising loop (1 full + N-1 cached steps), eager and as a CUDA graph
+    loop = None
+    if cfg.get("cached_steps", 0) > 1:
+        loop = time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops)
 
     # ---- end to end through the C ABI with host buffers (copies timed)
     h2d = sum(x.numel() * x.element_size() for x in host)
@@ -342,9 +390,11 @@ def run_ours(args, world, rank, local):
                    "step": "positions + full block-causal step with cache store + one cached step",
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "dp%d (independent requests per GPU)" % world},
-        "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps},
+        "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps,
+                      "ms_median": pct(full_each, 50), "ms_p95": pct(full_each, 95)},
         "cached_step": {"tflops": cached_tf, "frac_of_peak": cached_tf / peak,
-                        "ms": cached_ms / args.steps},
+                        "ms": cached_ms / args.steps, "ms_median": pct(cached_each, 50),
+                        "ms_p95": pct(cached_each, 95)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": ncu_traffic(name), "traffic_unit": "bytes/launch",
                      "kernel": "qi21::tc::attn_tc_kernel (full + cached launches)",
@@ -355,6 +405,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if loop is not None:
+        line["loop"] = loop
     print(json.dumps(line), flush=True)
 
 
@@ -362,7 +414,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="t2i", choices=[n for n in W.WORKLOADS if n != "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
