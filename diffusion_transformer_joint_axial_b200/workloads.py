@@ -101,6 +101,19 @@ def cached_inputs(name, step=2):
     return tuple(x[:, P:].contiguous() for x in (q, k, v))
 
 
+# QK-RMSNorm inputs.  The pages publish no trained weights, so the two
+# per-dimension weight vectors (queries, keys) are seeded synthetic values
+# around 1; eps is the 1e-6 the pages print for the model's other RMSNorms.
+QK_NORM_EPS = 1e-6
+
+
+def qk_norm_weights(seed=7):
+    """(w_q, w_k): float32 CPU tensors of 128 weights each, 1 + 0.25 * N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    return tuple(torch.from_numpy((1.0 + 0.25 * rng.standard_normal(HEAD_DIM)).astype(np.float32))
+                 for _ in range(2))
+
+
 def as_f64(t):
     """float64 numpy copy of a (CPU) torch tensor, for the oracle."""
     return t.detach().to("cpu").to(torch.float64).numpy()

@@ -35,6 +35,14 @@ What it computes (sources are the pages this build follows):
   over [cached prefix K/V || fresh target K/V] with no mask, since the target
   sees everything (overview, card 6A and learning goals).
 
+* ``rms_norm`` -- the QK-RMSNorm in front of RoPE: every head's 128-dim
+  query and key vector of every token is divided by its root mean square (plus
+  eps under the root) and multiplied by a learned per-dimension weight, one
+  weight vector for queries and one for keys, before the rotation ("Qwen-Image-2.1"
+  overview, card 4A; close reading, section 6: ``norm_q``/``norm_k`` are
+  RMSNorm(head_dim = 128) applied before ``apply_rope``).  The pages print no eps
+  for these two norms; callers pass it (the model's other RMSNorms use 1e-6).
+
 Inputs are arrays already cast to the GPU dtype (bf16 or fp32) by the seeded
 input module; every function promotes them to float64 first.
 
@@ -144,6 +152,19 @@ def rope(x, pos):
     out[:, 0::2] = x0 * c - x1 * s
     out[:, 1::2] = x0 * s + x1 * c
     return out
+
+
+# ----------------------------------------------------------------------------
+# QK-RMSNorm (applied to Q and K before the rotation)
+# ----------------------------------------------------------------------------
+
+def rms_norm(x, weight, eps):
+    """RMSNorm over the last axis (head_dim 128): x / sqrt(mean(x^2) + eps) * weight."""
+    x = np.asarray(x, dtype=np.float64)
+    weight = np.asarray(weight, dtype=np.float64)
+    assert x.shape[-1] == HEAD_DIM and weight.shape == (HEAD_DIM,)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * weight
 
 
 # ----------------------------------------------------------------------------

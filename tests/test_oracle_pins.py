@@ -262,11 +262,39 @@ def check_cached_equals_full(O):
     assert np.max(np.abs(cached - full[:, P:])) < 1e-13
 
 
+# ----------------------------------------------------------------- QK-norm --
+
+def check_rms_norm_vs_torch(O):
+    """Card 4A / close reading 6: norm_q and norm_k are RMSNorm(128) with a
+    weight; against torch's own rms_norm in float64."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((3, 5, 128)) * rng.uniform(0.05, 20.0, (3, 5, 1))
+    w = 1.0 + 0.25 * rng.standard_normal(128)
+    for eps in (1e-6, 0.5):
+        ref = torch.nn.functional.rms_norm(torch.tensor(x), (128,), torch.tensor(w), eps).numpy()
+        assert np.max(np.abs(O.rms_norm(x, w, eps) - ref)) < 1e-12
+
+
+def check_rms_norm_closed_forms(O):
+    """Constant rows, unit mean square, scale invariance, per-dimension weight."""
+    ones = np.ones(128)
+    for c in (3.0, -0.25):
+        y = O.rms_norm(np.full((1, 128), c), ones, 1e-6)
+        assert np.allclose(y, c / math.sqrt(c * c + 1e-6), rtol=1e-15, atol=0)
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((6, 128)) * 4.0
+    y = O.rms_norm(x, ones, 0.0)
+    assert np.allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-14, atol=0)
+    assert np.allclose(O.rms_norm(7.5 * x, ones, 0.0), y, rtol=1e-14, atol=1e-15)
+    w = rng.uniform(0.5, 2.0, 128)
+    assert np.allclose(O.rms_norm(x, w, 1e-6), O.rms_norm(x, ones, 1e-6) * w, rtol=1e-15, atol=0)
+
+
 CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_frames,
           check_prompt_length_invariance, check_block_causal_rule, check_prefix_never_sees_target,
           check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
           check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
-          check_cached_equals_full]
+          check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
@@ -357,6 +385,20 @@ def _head_v_transposed(q_rot, k_rot, v, kv_end=None, chunk=512):
     return OM.attention_head(q_rot, k_rot, v[::-1], kv_end, chunk)
 
 
+def _rms_sum_not_mean(x, weight, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * weight
+
+
+def _rms_eps_outside(x, weight, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps) * weight
+
+
+def _rms_no_weight(x, weight, eps):
+    return OM.rms_norm(x, np.ones(128), eps)
+
+
 MUTANTS = {
     "rope_sign": dict(rope=_rope_sign_flipped),
     "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
@@ -365,6 +407,9 @@ MUTANTS = {
     "text_mask_exclusive": dict(positions=_positions_text_exclusive),
     "missing_scale": dict(attention_head=_head_no_scale),
     "value_order": dict(attention_head=_head_v_transposed),
+    "rms_sum_not_mean": dict(rms_norm=_rms_sum_not_mean),
+    "rms_eps_outside_root": dict(rms_norm=_rms_eps_outside),
+    "rms_weight_dropped": dict(rms_norm=_rms_no_weight),
 }
 
 
