@@ -283,6 +283,7 @@ def run_ours(args, world, rank, local):
     ws_c = qi.new_workspace(qi.cached_workspace_size(B, H, P, T, dt), dev)
     pos = torch.empty((L, 3), dtype=torch.int32, device=dev)
     kv_end = torch.empty((L,), dtype=torch.int32, device=dev)
+    assert pos[P:].data_ptr() % 16 == 0, "target rows of the position table must be 16-byte aligned"
     seg_arr = qi._binding.to_segments(segs)
     lib = qi.load_library()
     stream = torch.cuda.current_stream(dev)
@@ -290,17 +291,25 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     P_ = qi._binding._ptr
 
+    if args.qk_norm:  # the fused QK-RMSNorm variant of both steps
+        wq, wk = (w.to(dev) for w in W.qk_norm_weights())
+        norm = (P_(wq), P_(wk), qi._binding.ctypes.c_float(W.QK_NORM_EPS))
+        full_fn = lambda *a: lib.qi21_attn_full_qknorm(*a[:13], *norm, *a[13:])
+        cached_fn = lambda *a: lib.qi21_attn_cached_qknorm(*a[:12], *norm, *a[12:])
+    else:
+        full_fn, cached_fn = lib.qi21_attn_full, lib.qi21_attn_cached
+
     def one_step(ev=None, qq=dq, kk=dk, vv=dv, qqt=dqt, kkt=dkt, vvt=dvt):
         lib.qi21_rope_positions(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
         if ev is not None:
             qi.time_next_attention(ev[0], ev[1])
-        st = lib.qi21_attn_full(B, H, L, P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
-                                P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
+        st = full_fn(B, H, L, P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
+                     P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
         assert st == 0, lib.qi21_last_error()
         if ev is not None:
             qi.time_next_attention(ev[2], ev[3])
-        st = lib.qi21_attn_cached(B, H, P, T, 0, P_(qqt), P_(kkt), P_(vvt), P_(pos[P:]), P_(kc), P_(vc),
-                                  P_(o_c), P_(ws_c), ws_c.numel(), sp)
+        st = cached_fn(B, H, P, T, 0, P_(qqt), P_(kkt), P_(vvt), P_(pos[P:]), P_(kc), P_(vc),
+                       P_(o_c), P_(ws_c), ws_c.numel(), sp)
         assert st == 0, lib.qi21_last_error()
 
     full_flops, cached_flops = step_flops(name)
@@ -334,7 +343,7 @@ def run_ours(args, world, rank, local):
 
     # ---- the denoising loop (1 full + N-1 cached steps), eager and as a CUDA graph
     loop = None
-    if cfg.get("cached_steps", 0) > 1:
+    if cfg.get("cached_steps", 0) > 1 and not args.qk_norm:
         loop = time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops)
 
     # ---- end to end through the C ABI with host buffers (copies timed)
@@ -387,7 +396,9 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": step_ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": W.DESCRIPTIONS[name], "B": B, "H": H, "L": L, "P": P, "T": T,
-                   "step": "positions + full block-causal step with cache store + one cached step",
+                   "step": "positions + full block-causal step with cache store + one cached step"
+                           + (", QK-RMSNorm fused (synthetic weights)" if args.qk_norm else ""),
+                   "qk_norm": bool(args.qk_norm),
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "dp%d (independent requests per GPU)" % world},
         "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps,
@@ -419,6 +430,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qk-norm", action="store_true",
+                    help="time the variant with the QK-RMSNorm fused in front of RoPE")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -27,7 +27,8 @@ WORKSPACE_HEADER_BYTES = 256
 EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_full",
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
-            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2")
+            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
+            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm")
 
 
 class QI21Error(RuntimeError):
@@ -66,6 +67,10 @@ def load_library(path=LIB_PATH):
     L.qi21_attn_cached_workspace_size.restype = _sz
     L.qi21_attn_cached.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _sz, _vp]
+    L.qi21_attn_full_qknorm.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
+    L.qi21_attn_cached_qknorm.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
     L.qi21_workspace_status.argtypes = [_vp, _vp]
     L.qi21_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
     L.qi21_status_string.argtypes = [_i32]
@@ -81,8 +86,8 @@ def load_library(path=LIB_PATH):
     L.qi21_attn_cached_noalloc.restype = _i32
     L.qi21_selftest_exp2.argtypes = [_vp, _vp, _i64, _vp]
     L.qi21_selftest_exp2.restype = _i32
-    for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached",
-                 "qi21_workspace_status", "qi21_selftest_wait_timeout"):
+    for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached", "qi21_attn_full_qknorm",
+                 "qi21_attn_cached_qknorm", "qi21_workspace_status", "qi21_selftest_wait_timeout"):
         getattr(L, name).restype = _i32
     _lib = L
     return L
@@ -176,11 +181,24 @@ def alloc_cache(B, H, P, dtype, device):
             torch.empty((B, H, P, HEAD_DIM), dtype=dtype, device=device))
 
 
-def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=None, workspace=None):
+def _norm_args(qk_norm, device):
+    """(w_q, w_k, eps) -> pointers and eps for the *_qknorm entry points."""
+    if qk_norm is None:
+        return None
+    w_q, w_k, eps = qk_norm
+    _need(w_q, "w_q", (HEAD_DIM,), torch.float32, device)
+    _need(w_k, "w_k", (HEAD_DIM,), torch.float32, device)
+    return _ptr(w_q), _ptr(w_k), ctypes.c_float(float(eps))
+
+
+def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=None, workspace=None,
+              qk_norm=None):
     """First step: block-causal joint attention; stores the prefix K/V cache if given.
 
     q, k, v: [B, L, H, 128] bf16 or fp32 on one CUDA device; pos [L, 3],
-    kv_end [L] int32 from :func:`rope_positions`.  Returns ``out``.
+    kv_end [L] int32 from :func:`rope_positions`.  ``qk_norm = (w_q, w_k, eps)``
+    (float32 [128] weights on the same device) fuses the QK-RMSNorm in front of
+    the rotation.  Returns ``out``.
     """
     L_ = _cuda_lib()
     B, L, H, D = q.shape
@@ -202,17 +220,26 @@ def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=
     need = full_workspace_size(B, H, L, P, dt)
     if workspace is None:
         workspace = new_workspace(need, dev)
+    norm = _norm_args(qk_norm, dev)
     with torch.cuda.device(dev):
-        _check(L_.qi21_attn_full(B, H, L, P, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(kv_end),
-                                 _ptr(out), _ptr(k_cache), _ptr(v_cache), _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream(dev)))
+        if norm is None:
+            _check(L_.qi21_attn_full(B, H, L, P, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(kv_end),
+                                     _ptr(out), _ptr(k_cache), _ptr(v_cache), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(dev)))
+        else:
+            _check(L_.qi21_attn_full_qknorm(B, H, L, P, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos),
+                                            _ptr(kv_end), _ptr(out), _ptr(k_cache), _ptr(v_cache), *norm,
+                                            _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                            _stream(dev)))
     return out
 
 
-def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None):
+def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk_norm=None):
     """Later step: target queries over [cached prefix K/V || fresh target K/V], no mask.
 
     q, k, v: [B, T, H, 128]; pos_tgt [T, 3]; k_cache, v_cache [B, H, P, 128].
+    ``qk_norm`` as for :func:`attn_full` (the cache must come from a full step
+    with the same norm).
     """
     L_ = _cuda_lib()
     B, T, H, D = q.shape
@@ -230,10 +257,17 @@ def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None):
     need = cached_workspace_size(B, H, P, T, dt)
     if workspace is None:
         workspace = new_workspace(need, dev)
+    norm = _norm_args(qk_norm, dev)
     with torch.cuda.device(dev):
-        _check(L_.qi21_attn_cached(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_tgt),
-                                   _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
-                                   workspace.numel() * workspace.element_size(), _stream(dev)))
+        if norm is None:
+            _check(L_.qi21_attn_cached(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_tgt),
+                                       _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(dev)))
+        else:
+            _check(L_.qi21_attn_cached_qknorm(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_tgt),
+                                              _ptr(k_cache), _ptr(v_cache), _ptr(out), *norm,
+                                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                              _stream(dev)))
     return out
 
 

@@ -78,6 +78,15 @@ static qi21_status check_ptr(const void* p, const char* name) {
     if (_s != QI21_OK) return _s;          \
   } while (0)
 
+// QK-RMSNorm arguments: both weight vectors or neither; eps finite, >= 0.
+static qi21_status check_norm(const float* norm_q, const float* norm_k, float eps) {
+  if (norm_q == nullptr && norm_k == nullptr) return QI21_OK;
+  QI21_TRY(check_ptr(norm_q, "norm_q"));
+  QI21_TRY(check_ptr(norm_k, "norm_k"));
+  if (!(eps >= 0.f) || !(eps < 3.0e38f)) return fail(QI21_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  return QI21_OK;
+}
+
 // Runs the attention kernel that matches the dtype.
 static qi21_status run_attention(const AttnArgs& a, qi21_dtype dt, cudaStream_t st) {
   cudaEvent_t t0 = g_time_start, t1 = g_time_stop;
@@ -152,10 +161,11 @@ size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t 
   return ws_layout(B, H, T, dt).total;
 }
 
-qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt, const void* q,
-                           const void* k, const void* v, const int32_t* pos, const int32_t* kv_end,
-                           void* o, void* k_cache, void* v_cache, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
+                                  const void* q, const void* k, const void* v, const int32_t* pos,
+                                  const int32_t* kv_end, void* o, void* k_cache, void* v_cache,
+                                  const float* norm_q, const float* norm_k, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
   QI21_TRY(check_common(B, H, dt));
   if (L < 0 || L > (int64_t)1 << 30) return fail(QI21_ERR_INVALID_ARG, "L out of range (%lld)", (long long)L);
   if (P < 0 || P > L) return fail(QI21_ERR_INVALID_ARG, "P must be in [0, L] (P=%lld, L=%lld)", (long long)P, (long long)L);
@@ -175,6 +185,7 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
   QI21_TRY(check_ptr(workspace, "workspace"));
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  QI21_TRY(check_norm(norm_q, norm_k, eps));
   const WsLayout w = ws_layout(B, H, L, dt);
   if (workspace_bytes < w.total)
     return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
@@ -201,6 +212,8 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
   rp.table = table;
   rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
+  rp.k_norm_w = norm_k;
+  rp.norm_eps = eps;
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
@@ -225,13 +238,16 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
                   kHeadDim, L * tokstride};
   a.o = o;
   a.status = status;
+  a.q_norm_w = norm_q;
+  a.norm_eps = eps;
   return run_attention(a, dt, st);
 }
 
-qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt, const void* q,
-                             const void* k, const void* v, const int32_t* pos_tgt, const void* k_cache,
-                             const void* v_cache, void* o, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                    const void* q, const void* k, const void* v,
+                                    const int32_t* pos_tgt, const void* k_cache, const void* v_cache,
+                                    void* o, const float* norm_q, const float* norm_k, float eps,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   QI21_TRY(check_common(B, H, dt));
   if (P < 0 || T < 0 || P > (int64_t)1 << 30 || T > (int64_t)1 << 30)
     return fail(QI21_ERR_INVALID_ARG, "P and T must be in [0, 2^30] (P=%lld, T=%lld)", (long long)P, (long long)T);
@@ -248,6 +264,7 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
   QI21_TRY(check_ptr(workspace, "workspace"));
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  QI21_TRY(check_norm(norm_q, norm_k, eps));
   const WsLayout w = ws_layout(B, H, T, dt);
   if (workspace_bytes < w.total)
     return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
@@ -270,6 +287,8 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
   rp.table = table;
   rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
+  rp.k_norm_w = norm_k;
+  rp.norm_eps = eps;
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
@@ -289,7 +308,47 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
   a.v1 = KvSource{v, T, tokstride, kHeadDim, T * tokstride};
   a.o = o;
   a.status = status;
+  a.q_norm_w = norm_q;
+  a.norm_eps = eps;
   return run_attention(a, dt, st);
+}
+
+qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt, const void* q,
+                           const void* k, const void* v, const int32_t* pos, const int32_t* kv_end,
+                           void* o, void* k_cache, void* v_cache, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return attn_full_impl(B, H, L, P, dt, q, k, v, pos, kv_end, o, k_cache, v_cache, nullptr, nullptr,
+                        0.f, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_attn_full_qknorm(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
+                                  const void* q, const void* k, const void* v, const int32_t* pos,
+                                  const int32_t* kv_end, void* o, void* k_cache, void* v_cache,
+                                  const float* norm_q, const float* norm_k, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (norm_q == nullptr || norm_k == nullptr)
+    return fail(QI21_ERR_INVALID_ARG, "norm_q and norm_k must be given");
+  return attn_full_impl(B, H, L, P, dt, q, k, v, pos, kv_end, o, k_cache, v_cache, norm_q, norm_k,
+                        eps, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt, const void* q,
+                             const void* k, const void* v, const int32_t* pos_tgt, const void* k_cache,
+                             const void* v_cache, void* o, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return attn_cached_impl(B, H, P, T, dt, q, k, v, pos_tgt, k_cache, v_cache, o, nullptr, nullptr,
+                          0.f, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                    const void* q, const void* k, const void* v,
+                                    const int32_t* pos_tgt, const void* k_cache, const void* v_cache,
+                                    void* o, const float* norm_q, const float* norm_k, float eps,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (norm_q == nullptr || norm_k == nullptr)
+    return fail(QI21_ERR_INVALID_ARG, "norm_q and norm_k must be given");
+  return attn_cached_impl(B, H, P, T, dt, q, k, v, pos_tgt, k_cache, v_cache, o, norm_q, norm_k, eps,
+                          workspace, workspace_bytes, stream);
 }
 
 qi21_status qi21_workspace_status(void* workspace, void* stream) {

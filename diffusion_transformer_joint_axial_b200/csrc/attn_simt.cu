@@ -2,8 +2,8 @@
 // dense tensor-core path that meets a 1e-4 bound in one pass).
 //
 // One CTA = 16 query rows of one (batch, head); 8 warps x 2 rows.  The query
-// rows are rotated on load with the per-token (cos, sin) table; keys arrive
-// already rotated.  Key tiles of 32 that lie at or beyond the largest
+// rows are rotated on load with the per-token (cos, sin) table (after the
+// QK-RMSNorm, when its weight is given); keys arrive already rotated.  Key tiles of 32 that lie at or beyond the largest
 // visibility bound of the CTA's rows are never loaded (block-causal skip);
 // inside the loaded tiles each row masks keys j >= kv_end[i].  Online softmax
 // in fp32 with expf.
@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kSimtThreads)
   __shared__ float sk[kSimtKeys][kHeadDim + 1];
   __shared__ float sv[kSimtKeys][kHeadDim];
   __shared__ int s_kvhi;
+  __shared__ float s_rs[kSimtRows];  // QK-RMSNorm: rsqrt(mean square + eps) of each query row
 
   const int b = blockIdx.z, h = blockIdx.y;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kSimtRows;
@@ -37,6 +38,24 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int64_t tok_stride = static_cast<int64_t>(a.H) * kHeadDim;
   const float* q = static_cast<const float*>(a.q);
 
+  // QK-RMSNorm of the query rows (when a weight is given): one warp per row,
+  // four elements per lane, a shuffle sum
+  const bool norm = a.q_norm_w != nullptr;
+  if (norm) {
+    for (int r = warp; r < kSimtRows; r += kSimtThreads / 32) {
+      const int64_t row = row0 + r;
+      float ss = 0.f;
+      if (row < a.Lq) {
+        const float4 x = *reinterpret_cast<const float4*>(q + (b * a.Lq + row) * tok_stride +
+                                                          h * kHeadDim + 4 * lane);
+        ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) s_rs[r] = rsqrtf(ss * (1.f / kHeadDim) + a.norm_eps);
+    }
+    __syncthreads();
+  }
   // rotated query rows
   for (int e = threadIdx.x; e < kSimtRows * (kHeadDim / 2); e += blockDim.x) {
     const int r = e / (kHeadDim / 2), m = e % (kHeadDim / 2);
@@ -45,8 +64,13 @@ __global__ void __launch_bounds__(kSimtThreads)
     if (row < a.Lq) {
       const float* src = q + (b * a.Lq + row) * tok_stride + h * kHeadDim + 2 * m;
       const float2 cs = a.table[row * kPairs + m];
-      y0 = fmaf(src[0], cs.x, -src[1] * cs.y);
-      y1 = fmaf(src[0], cs.y, src[1] * cs.x);
+      float x0 = src[0], x1 = src[1];
+      if (norm) {
+        x0 *= s_rs[r] * a.q_norm_w[2 * m];
+        x1 *= s_rs[r] * a.q_norm_w[2 * m + 1];
+      }
+      y0 = fmaf(x0, cs.x, -x1 * cs.y);
+      y1 = fmaf(x0, cs.y, x1 * cs.x);
     }
     sq[r][2 * m] = y0;
     sq[r][2 * m + 1] = y1;

@@ -92,6 +92,8 @@ struct Params {
   __nv_bfloat16* o;
   uint32_t* status;
   uint32_t* unit_counter;  // zeroed by the pre-pass kernel before this launch
+  const float* q_norm_w;   // [128] QK-RMSNorm weight of Q, or null
+  float norm_eps;
 };
 
 constexpr int kSchedSlots = 4;
@@ -103,6 +105,7 @@ struct __align__(1024) Smem {
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   float row_l[2][2][BM];  // [unit parity][tile][row]: softmax -> epilogue
+  alignas(16) float qnw[kHeadDim];  // QK-RMSNorm weight of Q (when given)
   int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
   uint64_t q_full[2], q_rot[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
@@ -177,6 +180,49 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
     U.N[s] = tiles_below(p, kv_hi);
   }
   return U;
+}
+
+// QK-RMSNorm + rotation of one query row in its 128B-swizzled tile (row t):
+// the row's mean square (fp32, from the bf16 values), then each adjacent pair
+// (2m, 2m+1) scaled by rsqrt(mean square + eps) and the weight and rotated by
+// the token's (cos, sin), rounded once to bf16.
+__device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const float4* cs, int t,
+                                                  const float* wn, float eps) {
+  float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < 16; ++c) {
+    const int half = c >> 3, cc = c & 7;
+    const uint4 x = *reinterpret_cast<const uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v = unpack_bf16x2(w[e]);
+      ss0 = fmaf(v.x, v.x, ss0);
+      ss1 = fmaf(v.y, v.y, ss1);
+    }
+  }
+  const float rs = rsqrtf((ss0 + ss1) * (1.f / kHeadDim) + eps);
+#pragma unroll 2
+  for (int c = 0; c < 16; ++c) {
+    const int half = c >> 3, cc = c & 7;
+    uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
+    uint4 x = *ptr;
+    const float4 r01 = __ldg(cs + 2 * c);
+    const float4 r23 = __ldg(cs + 2 * c + 1);
+    const float4 w0 = *reinterpret_cast<const float4*>(wn + 8 * c);
+    const float4 w1 = *reinterpret_cast<const float4*>(wn + 8 * c + 4);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const float cv[4] = {r01.x, r01.z, r23.x, r23.z};
+    const float sv[4] = {r01.y, r01.w, r23.y, r23.w};
+    uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v = unpack_bf16x2(w[e]);
+      const float x0 = v.x * rs * wv[2 * e], x1 = v.y * rs * wv[2 * e + 1];
+      w[e] = pack_bf16x2(fmaf(x0, cv[e], -x1 * sv[e]), fmaf(x0, sv[e], x1 * cv[e]));
+    }
+    *ptr = x;
+  }
 }
 
 // Key tile n: first key index j0 (in the joint key order), key count, source
@@ -326,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
     tmem_relinquish();
   }
+  if (p.q_norm_w != nullptr && threadIdx.x < kHeadDim) S.qnw[threadIdx.x] = p.q_norm_w[threadIdx.x];
   if (warp == kWarpLoad && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k0);
@@ -604,23 +651,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (valid) {
         const float4* cs = reinterpret_cast<const float4*>(p.table + (size_t)row * kPairs);
         uint8_t* qrow = S.q[s] + t * 128;
+        if (p.q_norm_w == nullptr) {
 #pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-          const int half = c >> 3, cc = c & 7;
-          uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
-          uint4 x = *ptr;
-          const float4 r01 = __ldg(cs + 2 * c);
-          const float4 r23 = __ldg(cs + 2 * c + 1);
-          uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-          float2 xv = unpack_bf16x2(w[0]);
-          w[0] = pack_bf16x2(fmaf(xv.x, r01.x, -xv.y * r01.y), fmaf(xv.x, r01.y, xv.y * r01.x));
-          xv = unpack_bf16x2(w[1]);
-          w[1] = pack_bf16x2(fmaf(xv.x, r01.z, -xv.y * r01.w), fmaf(xv.x, r01.w, xv.y * r01.z));
-          xv = unpack_bf16x2(w[2]);
-          w[2] = pack_bf16x2(fmaf(xv.x, r23.x, -xv.y * r23.y), fmaf(xv.x, r23.y, xv.y * r23.x));
-          xv = unpack_bf16x2(w[3]);
-          w[3] = pack_bf16x2(fmaf(xv.x, r23.z, -xv.y * r23.w), fmaf(xv.x, r23.w, xv.y * r23.z));
-          *ptr = x;
+          for (int c = 0; c < 16; ++c) {
+            const int half = c >> 3, cc = c & 7;
+            uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
+            uint4 x = *ptr;
+            const float4 r01 = __ldg(cs + 2 * c);
+            const float4 r23 = __ldg(cs + 2 * c + 1);
+            uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+            float2 xv = unpack_bf16x2(w[0]);
+            w[0] = pack_bf16x2(fmaf(xv.x, r01.x, -xv.y * r01.y), fmaf(xv.x, r01.y, xv.y * r01.x));
+            xv = unpack_bf16x2(w[1]);
+            w[1] = pack_bf16x2(fmaf(xv.x, r01.z, -xv.y * r01.w), fmaf(xv.x, r01.w, xv.y * r01.z));
+            xv = unpack_bf16x2(w[2]);
+            w[2] = pack_bf16x2(fmaf(xv.x, r23.x, -xv.y * r23.y), fmaf(xv.x, r23.y, xv.y * r23.x));
+            xv = unpack_bf16x2(w[3]);
+            w[3] = pack_bf16x2(fmaf(xv.x, r23.z, -xv.y * r23.w), fmaf(xv.x, r23.w, xv.y * r23.z));
+            *ptr = x;
+          }
+        } else {
+          norm_rotate_q_row(qrow, cs, t, S.qnw, p.norm_eps);
         }
       }
       fence_proxy_async_smem();
@@ -787,6 +838,8 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.status = a.status;
   p.unit_counter = a.unit_counter;
+  p.q_norm_w = a.q_norm_w;
+  p.norm_eps = a.norm_eps;
   const size_t smem = sizeof(tc::Smem) + 1024;
   cudaError_t err =
       cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -57,6 +57,9 @@ cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream) {
 // height axis, the rest the width axis ("3A", section 1: bands 16/56/56).
 // Every K row is rotated once here and stored head-major (the Prefix rows go
 // straight into the KV cache); V's prefix rows are copied into the V cache.
+// With a K norm weight, each head row is first divided by its root mean
+// square (plus eps under the root) and multiplied by the weight: the
+// QK-RMSNorm that precedes RoPE (overview card 4A; close reading section 6).
 
 Omega make_omega() {
   Omega o;
@@ -104,6 +107,46 @@ __device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float*)
   }
 }
 
+// Sum of squares of a 16-byte chunk.
+__device__ __forceinline__ float sumsq_chunk(const uint4& u, __nv_bfloat16*) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = unpack_bf16x2(w[e]);
+    s = fmaf(x.x, x.x, fmaf(x.y, x.y, s));
+  }
+  return s;
+}
+__device__ __forceinline__ float sumsq_chunk(const uint4& u, float*) {
+  const float* x = reinterpret_cast<const float*>(&u);
+  return fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], x[3] * x[3])));
+}
+
+// x * rs * weight, then the rotation, on one chunk (wt: the chunk's weights).
+__device__ __forceinline__ void norm_rotate_chunk(uint4& u, const float2* cs, float rs,
+                                                  const float* wt, __nv_bfloat16*) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 xr = unpack_bf16x2(w[e]);
+    const float x0 = xr.x * rs * wt[2 * e], x1 = xr.y * rs * wt[2 * e + 1];
+    const float2 r = cs[e];
+    w[e] = pack_bf16x2(fmaf(x0, r.x, -x1 * r.y), fmaf(x0, r.y, x1 * r.x));
+  }
+}
+__device__ __forceinline__ void norm_rotate_chunk(uint4& u, const float2* cs, float rs,
+                                                  const float* wt, float*) {
+  float* x = reinterpret_cast<float*>(&u);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float2 r = cs[e];
+    const float x0 = x[2 * e] * rs * wt[2 * e], x1 = x[2 * e + 1] * rs * wt[2 * e + 1];
+    x[2 * e] = fmaf(x0, r.x, -x1 * r.y);
+    x[2 * e + 1] = fmaf(x0, r.y, x1 * r.x);
+  }
+}
+
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -116,7 +159,10 @@ template <typename T>
 __global__ void __launch_bounds__(kPrepThreads)
     rope_prep_kernel(const __grid_constant__ RopePrepParams p) {
   __shared__ float2 cs[kPrepTokens][kPairs];
+  __shared__ __align__(16) float wn[kHeadDim];
   const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kPrepTokens;
+  const bool norm = p.k_norm_w != nullptr;
+  if (norm && threadIdx.x < kHeadDim) wn[threadIdx.x] = p.k_norm_w[threadIdx.x];
   const int b = blockIdx.y;
   if (p.unit_counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
     *p.unit_counter = 0u;
@@ -142,7 +188,12 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int items = ntok * H * CPR;
   const T* __restrict__ k = static_cast<const T*>(p.k);
   const T* __restrict__ v = static_cast<const T*>(p.v);
-  for (int e0 = threadIdx.x; e0 < items; e0 += kPrepUnroll * kPrepThreads) {
+  // The CPR chunks of one head row sit in CPR consecutive lanes of one warp
+  // (CPR divides 32 and the thread count): the norm's row sum is a shuffle
+  // reduction among them.  The loop runs while any lane of the warp has work,
+  // so every lane takes part in the shuffles.
+  const int lane = threadIdx.x & 31;
+  for (int e0 = threadIdx.x; e0 - lane < items; e0 += kPrepUnroll * kPrepThreads) {
     uint4 ku[kPrepUnroll], vu[kPrepUnroll];
     int64_t src[kPrepUnroll];
 #pragma unroll
@@ -161,13 +212,23 @@ __global__ void __launch_bounds__(kPrepThreads)
 #pragma unroll
     for (int i = 0; i < kPrepUnroll; ++i) {
       const int e = e0 + i * kPrepThreads;
+      float rs = 1.f;
+      if (norm) {
+        float ss = e < items ? sumsq_chunk(ku[i], static_cast<T*>(nullptr)) : 0.f;
+#pragma unroll
+        for (int o = CPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        rs = rsqrtf(ss * (1.f / kHeadDim) + p.norm_eps);
+      }
       if (e >= items) continue;
       const int t = e / (H * CPR);
       const int rem = e - t * (H * CPR);
       const int h = rem / CPR;
       const int c = rem - h * CPR;
       const int64_t tok = tok0 + t;
-      rotate_chunk(ku[i], &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
+      if (norm)
+        norm_rotate_chunk(ku[i], &cs[t][c * EPC / 2], rs, &wn[c * EPC], static_cast<T*>(nullptr));
+      else
+        rotate_chunk(ku[i], &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
       T* dst;
       int64_t row, rows;
       if (tok < p.split) {

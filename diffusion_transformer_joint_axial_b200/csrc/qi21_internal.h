@@ -60,6 +60,8 @@ struct RopePrepParams {
   float2* table;   // [Lk][64] (cos, sin) of every token, or null
   uint32_t* unit_counter;  // zeroed here for the attention launch that follows, or null
   Omega omega;
+  const float* k_norm_w;   // [128] QK-RMSNorm weight of K, or null (no norm)
+  float norm_eps;
 };
 cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream);
 
@@ -85,6 +87,8 @@ struct AttnArgs {
   void* o;                // token-major [B, Lq, H, 128]
   uint32_t* status;       // workspace header status word
   uint32_t* unit_counter; // workspace header: dynamic-schedule counter (zeroed by the pre-pass)
+  const float* q_norm_w;  // [128] QK-RMSNorm weight of Q, or null (no norm)
+  float norm_eps;
 };
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);

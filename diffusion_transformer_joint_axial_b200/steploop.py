@@ -45,7 +45,7 @@ class DenoiseLoop:
         D = qb.HEAD_DIM
         mk = lambda *shape: torch.zeros(shape, dtype=dtype, device=dev)
         self.pos, self.kv_end = qb.rope_positions(segments, dev)
-        self.pos_t = self.pos[self.P:].contiguous()
+        self.pos_t = self.pos[self.P:].clone()  # own allocation: 16-byte aligned
         self.q, self.k, self.v = (mk(B, self.L, H, D) for _ in range(3))
         n = steps - 1
         self.target_q, self.target_k, self.target_v = (

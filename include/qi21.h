@@ -150,6 +150,38 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
                              void* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qi21_attn_full_qknorm / qi21_attn_cached_qknorm -- the same two steps with
+ * the QK-RMSNorm that precedes RoPE fused in (overview card 4A "Single-Stream
+ * DiT Attention & QK-RMSNorm"; close reading section 6: norm_q and norm_k are
+ * RMSNorm(head_dim = 128), applied to every head of every token before the
+ * rotation).  Each Q and K head vector x becomes
+ *     x / sqrt(mean(x^2) + eps) * w        (w = norm_q for Q, norm_k for K),
+ * computed in fp32 from the stored values, then rotated and rounded once to
+ * the storage type.  V is not normalised.
+ *
+ *   norm_q, norm_k  device float32 [128] each (16-byte aligned), read; both
+ *                   must be given (QI21_ERR_INVALID_ARG otherwise).
+ *   eps             finite, >= 0 (the pages print 1e-6 for the model's other
+ *                   RMSNorms and none for these two).  An all-zero head row with
+ *                   eps = 0 divides by zero, as the formula does.
+ *   other arguments as for qi21_attn_full / qi21_attn_cached.
+ * The cache written by qi21_attn_full_qknorm holds normalised, rotated prefix K;
+ * use it with qi21_attn_cached_qknorm and the same norm_k.
+ */
+qi21_status qi21_attn_full_qknorm(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
+                                  const void* q, const void* k, const void* v,
+                                  const int32_t* pos, const int32_t* kv_end, void* o,
+                                  void* k_cache, void* v_cache,
+                                  const float* norm_q, const float* norm_k, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                    const void* q, const void* k, const void* v,
+                                    const int32_t* pos_tgt, const void* k_cache,
+                                    const void* v_cache, void* o,
+                                    const float* norm_q, const float* norm_k, float eps,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * qi21_attn_cached_noalloc -- the cached step of qi21_attn_cached for callers
  * that may not allocate device memory (plugin hosts that only hand over a
  * stream and tensors, servers that reserve all memory at start-up, loops where

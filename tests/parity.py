@@ -59,12 +59,13 @@ def gpu_cached(q_t, k_t, v_t, pos_t, kc, vc, device="cuda"):
     return o.cpu()
 
 
-def check_cache(kc, vc, k, v, pos, P, heads=None, batches=None):
+def check_cache(kc, vc, k, v, pos, P, heads=None, batches=None, k_f64=None):
     """GPU cache vs the oracle's step-1 store: V copied exactly, K rotated
-    within one rounding of the storage type."""
+    within one rounding of the storage type.  ``k_f64`` replaces the keys the
+    oracle rotates (the QK-normalised keys, for the fused norm)."""
     if P == 0:
         return
-    kf, vf = W.as_f64(k), W.as_f64(v)
+    kf, vf = (W.as_f64(k) if k_f64 is None else k_f64), W.as_f64(v)
     ok, ov = O.prefix_cache(kf, vf, pos, P, heads=heads, batches=batches)
     heads = list(range(k.shape[2])) if heads is None else list(heads)
     batches = list(range(k.shape[0])) if batches is None else list(batches)

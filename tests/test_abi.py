@@ -129,6 +129,24 @@ def test_attn_cached_rejects(lib):
     assert lib.qi21_attn_cached(*args(4, 0, p(16), p(256), 10)) == qb.QI21_OK  # T = 0: nothing to do
 
 
+def test_qknorm_rejects(lib):
+    p = ctypes.c_void_p
+    full = lambda nq, nk, eps: lib.qi21_attn_full_qknorm(
+        1, 2, 32, 16, qb.QI21_BF16, p(16), p(16), p(16), p(16), p(16), p(16), None, None, nq, nk,
+        ctypes.c_float(eps), p(256), 1 << 30, None)
+    cached = lambda nq, nk, eps: lib.qi21_attn_cached_qknorm(
+        1, 2, 16, 16, qb.QI21_BF16, p(16), p(16), p(16), p(16), p(16), p(16), p(16), nq, nk,
+        ctypes.c_float(eps), p(256), 1 << 30, None)
+    for fn in (full, cached):
+        assert fn(None, p(16), 1e-6) == qb.QI21_ERR_INVALID_ARG      # weights missing
+        assert fn(p(16), None, 1e-6) == qb.QI21_ERR_INVALID_ARG
+        assert fn(p(16), p(20), 1e-6) == qb.QI21_ERR_INVALID_ARG     # misaligned weight
+        assert fn(p(16), p(16), -1.0) == qb.QI21_ERR_INVALID_ARG     # negative eps
+        assert fn(p(16), p(16), float("nan")) == qb.QI21_ERR_INVALID_ARG
+        assert fn(p(16), p(16), float("inf")) == qb.QI21_ERR_INVALID_ARG
+        assert "eps" in lib.qi21_last_error().decode()
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.qi21_selftest_wait_timeout(ctypes.c_void_p(256), 0, None) == qb.QI21_ERR_INVALID_ARG
 
