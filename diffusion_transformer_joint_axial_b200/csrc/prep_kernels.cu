@@ -60,6 +60,9 @@ cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream) {
 // With a K norm weight, each head row is first divided by its root mean
 // square (plus eps under the root) and multiplied by the weight: the
 // QK-RMSNorm that precedes RoPE (overview card 4A; close reading section 6).
+// Work split: a CTA takes four tokens of one batch; its K chunks are numbered
+// (token, head, chunk) and dealt to the threads round-robin, the first loads
+// going out before the float64 angles are computed.
 
 Omega make_omega() {
   Omega o;
@@ -70,7 +73,7 @@ Omega make_omega() {
   return o;
 }
 
-constexpr int kPrepTokens = 4;  // tokens per CTA: one (token, pair) angle per thread
+constexpr int kPrepTokens = 4;  // tokens per CTA
 constexpr int kPrepThreads = 256;
 constexpr int kPrepUnroll = 4;  // 16-byte loads each thread keeps in flight
 
@@ -84,28 +87,6 @@ template <>
 struct Vec16<float> {
   static constexpr int N = 4;
 };
-
-__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, __nv_bfloat16*) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 x = unpack_bf16x2(w[e]);
-    const float2 r = cs[e];
-    const float y0 = fmaf(x.x, r.x, -x.y * r.y);
-    const float y1 = fmaf(x.x, r.y, x.y * r.x);
-    w[e] = pack_bf16x2(y0, y1);
-  }
-}
-__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float*) {
-  float* x = reinterpret_cast<float*>(&u);
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float2 r = cs[e];
-    const float x0 = x[2 * e], x1 = x[2 * e + 1];
-    x[2 * e] = fmaf(x0, r.x, -x1 * r.y);
-    x[2 * e + 1] = fmaf(x0, r.y, x1 * r.x);
-  }
-}
 
 // Sum of squares of a 16-byte chunk.
 __device__ __forceinline__ float sumsq_chunk(const uint4& u, __nv_bfloat16*) {
@@ -123,25 +104,34 @@ __device__ __forceinline__ float sumsq_chunk(const uint4& u, float*) {
   return fmaf(x[0], x[0], fmaf(x[1], x[1], fmaf(x[2], x[2], x[3] * x[3])));
 }
 
-// x * rs * weight, then the rotation, on one chunk (wt: the chunk's weights).
-__device__ __forceinline__ void norm_rotate_chunk(uint4& u, const float2* cs, float rs,
-                                                  const float* wt, __nv_bfloat16*) {
+// (x * scale * weight), then the rotation by the pairs' (cos, sin), on one
+// chunk; wt is null when there is no norm (scale is then 1).
+__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float scale, const float* wt,
+                                             __nv_bfloat16*) {
   uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const float2 xr = unpack_bf16x2(w[e]);
-    const float x0 = xr.x * rs * wt[2 * e], x1 = xr.y * rs * wt[2 * e + 1];
+    float x0 = xr.x, x1 = xr.y;
+    if (wt != nullptr) {
+      x0 *= scale * wt[2 * e];
+      x1 *= scale * wt[2 * e + 1];
+    }
     const float2 r = cs[e];
     w[e] = pack_bf16x2(fmaf(x0, r.x, -x1 * r.y), fmaf(x0, r.y, x1 * r.x));
   }
 }
-__device__ __forceinline__ void norm_rotate_chunk(uint4& u, const float2* cs, float rs,
-                                                  const float* wt, float*) {
+__device__ __forceinline__ void rotate_chunk(uint4& u, const float2* cs, float scale, const float* wt,
+                                             float*) {
   float* x = reinterpret_cast<float*>(&u);
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
+    float x0 = x[2 * e], x1 = x[2 * e + 1];
+    if (wt != nullptr) {
+      x0 *= scale * wt[2 * e];
+      x1 *= scale * wt[2 * e + 1];
+    }
     const float2 r = cs[e];
-    const float x0 = x[2 * e] * rs * wt[2 * e], x1 = x[2 * e + 1] * rs * wt[2 * e + 1];
     x[2 * e] = fmaf(x0, r.x, -x1 * r.y);
     x[2 * e + 1] = fmaf(x0, r.y, x1 * r.x);
   }
@@ -155,20 +145,59 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
+// One 16-byte chunk of the work: token t of the CTA, head h, chunk c of the
+// head row.  The chunks of one row are CPR consecutive work items, so they
+// sit in CPR consecutive lanes.
+struct PrepItem {
+  int t, h, c;
+};
+template <int CPR>
+__device__ __forceinline__ PrepItem prep_item(int e, int H, float inv_h) {
+  PrepItem it;
+  const int r = e / CPR;  // row (t, h); CPR is a power of two
+  it.c = e - r * CPR;
+  // r / H through the reciprocal: exact for the few rows of one CTA
+  it.t = static_cast<int>((static_cast<float>(r) + 0.5f) * inv_h);
+  it.h = r - it.t * H;
+  return it;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kPrepThreads)
     rope_prep_kernel(const __grid_constant__ RopePrepParams p) {
   __shared__ float2 cs[kPrepTokens][kPairs];
-  __shared__ __align__(16) float wn[kHeadDim];
+  __shared__ __align__(16) float wn[kHeadDim];  // norm weight of K
+  constexpr int EPC = Vec16<T>::N;     // elements per 16-byte chunk
+  constexpr int CPR = kHeadDim / EPC;  // chunks per head row
   const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kPrepTokens;
-  const bool norm = p.k_norm_w != nullptr;
-  if (norm && threadIdx.x < kHeadDim) wn[threadIdx.x] = p.k_norm_w[threadIdx.x];
   const int b = blockIdx.y;
+  const int lane = threadIdx.x & 31;
   if (p.unit_counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
     *p.unit_counter = 0u;
   const int ntok = static_cast<int>(p.Lk - tok0 < kPrepTokens ? p.Lk - tok0 : kPrepTokens);
+  const int H = p.H;
+  const int items = ntok * H * CPR;
+  const float inv_h = 1.0f / static_cast<float>(H);
+  const bool norm = p.k_norm_w != nullptr;
+  const T* __restrict__ k = static_cast<const T*>(p.k);
 
-  {
+  // The first loads go out before the angles are computed: they do not need them.
+  uint4 x[kPrepUnroll];
+  auto issue = [&](int e0) {
+#pragma unroll
+    for (int i = 0; i < kPrepUnroll; ++i) {
+      const int e = e0 + i * kPrepThreads;
+      if (e < items) {
+        const PrepItem it = prep_item<CPR>(e, H, inv_h);
+        x[i] = ld_stream(k + ((static_cast<int64_t>(b) * p.Lk + tok0 + it.t) * H + it.h) * kHeadDim +
+                         it.c * EPC);
+      }
+    }
+  };
+  issue(threadIdx.x);
+
+  if (norm && threadIdx.x < kHeadDim) wn[threadIdx.x] = p.k_norm_w[threadIdx.x];
+  if (threadIdx.x < kPrepTokens * kPairs) {
     const int t = threadIdx.x / kPairs, m = threadIdx.x % kPairs;
     if (t < ntok) {
       const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
@@ -182,53 +211,26 @@ __global__ void __launch_bounds__(kPrepThreads)
   }
   __syncthreads();
 
-  constexpr int EPC = Vec16<T>::N;     // elements per 16-byte chunk
-  constexpr int CPR = kHeadDim / EPC;  // chunks per head row
-  const int H = p.H;
-  const int items = ntok * H * CPR;
-  const T* __restrict__ k = static_cast<const T*>(p.k);
-  const T* __restrict__ v = static_cast<const T*>(p.v);
-  // The CPR chunks of one head row sit in CPR consecutive lanes of one warp
-  // (CPR divides 32 and the thread count): the norm's row sum is a shuffle
-  // reduction among them.  The loop runs while any lane of the warp has work,
-  // so every lane takes part in the shuffles.
-  const int lane = threadIdx.x & 31;
+  // The loop runs while any lane of the warp has work, so that every lane
+  // takes part in the norm's shuffle reduction (a row's CPR chunks are CPR
+  // consecutive lanes: CPR divides 32 and the thread count).
   for (int e0 = threadIdx.x; e0 - lane < items; e0 += kPrepUnroll * kPrepThreads) {
-    uint4 ku[kPrepUnroll], vu[kPrepUnroll];
-    int64_t src[kPrepUnroll];
-#pragma unroll
-    for (int i = 0; i < kPrepUnroll; ++i) {
-      const int e = e0 + i * kPrepThreads;
-      if (e < items) {
-        const int t = e / (H * CPR);
-        const int rem = e - t * (H * CPR);
-        const int h = rem / CPR;
-        const int c = rem - h * CPR;
-        src[i] = ((static_cast<int64_t>(b) * p.Lk + tok0 + t) * H + h) * kHeadDim + c * EPC;
-        ku[i] = ld_stream(k + src[i]);
-        if (p.v_dst0 != nullptr && tok0 + t < p.split) vu[i] = ld_stream(v + src[i]);
-      }
-    }
+    if (e0 != static_cast<int>(threadIdx.x)) issue(e0);
 #pragma unroll
     for (int i = 0; i < kPrepUnroll; ++i) {
       const int e = e0 + i * kPrepThreads;
       float rs = 1.f;
       if (norm) {
-        float ss = e < items ? sumsq_chunk(ku[i], static_cast<T*>(nullptr)) : 0.f;
+        float ss = e < items ? sumsq_chunk(x[i], static_cast<T*>(nullptr)) : 0.f;
 #pragma unroll
         for (int o = CPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         rs = rsqrtf(ss * (1.f / kHeadDim) + p.norm_eps);
       }
       if (e >= items) continue;
-      const int t = e / (H * CPR);
-      const int rem = e - t * (H * CPR);
-      const int h = rem / CPR;
-      const int c = rem - h * CPR;
-      const int64_t tok = tok0 + t;
-      if (norm)
-        norm_rotate_chunk(ku[i], &cs[t][c * EPC / 2], rs, &wn[c * EPC], static_cast<T*>(nullptr));
-      else
-        rotate_chunk(ku[i], &cs[t][c * EPC / 2], static_cast<T*>(nullptr));
+      const PrepItem it = prep_item<CPR>(e, H, inv_h);
+      const int64_t tok = tok0 + it.t;
+      rotate_chunk(x[i], &cs[it.t][it.c * EPC / 2], rs, norm ? &wn[it.c * EPC] : nullptr,
+                   static_cast<T*>(nullptr));
       T* dst;
       int64_t row, rows;
       if (tok < p.split) {
@@ -240,10 +242,37 @@ __global__ void __launch_bounds__(kPrepThreads)
         row = tok - p.split;
         rows = p.Lk - p.split;
       }
-      const int64_t dsti = ((static_cast<int64_t>(b) * H + h) * rows + row) * kHeadDim + c * EPC;
-      *reinterpret_cast<uint4*>(dst + dsti) = ku[i];
-      if (p.v_dst0 != nullptr && tok < p.split)
-        *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) + dsti) = vu[i];
+      *reinterpret_cast<uint4*>(dst + ((static_cast<int64_t>(b) * H + it.h) * rows + row) * kHeadDim +
+                                it.c * EPC) = x[i];
+    }
+  }
+
+  // Prefix V rows: a plain copy into the V cache.
+  if (p.v_dst0 != nullptr && tok0 < p.split) {
+    const int nv = static_cast<int>(p.split - tok0 < ntok ? p.split - tok0 : ntok);
+    const int vitems = nv * H * CPR;
+    const T* __restrict__ v = static_cast<const T*>(p.v);
+    for (int e0 = threadIdx.x; e0 < vitems; e0 += kPrepUnroll * kPrepThreads) {
+      uint4 y[kPrepUnroll];
+#pragma unroll
+      for (int i = 0; i < kPrepUnroll; ++i) {
+        const int e = e0 + i * kPrepThreads;
+        if (e < vitems) {
+          const PrepItem it = prep_item<CPR>(e, H, inv_h);
+          y[i] = ld_stream(v + ((static_cast<int64_t>(b) * p.Lk + tok0 + it.t) * H + it.h) * kHeadDim +
+                           it.c * EPC);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kPrepUnroll; ++i) {
+        const int e = e0 + i * kPrepThreads;
+        if (e < vitems) {
+          const PrepItem it = prep_item<CPR>(e, H, inv_h);
+          *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) +
+                                    ((static_cast<int64_t>(b) * H + it.h) * p.split + tok0 + it.t) * kHeadDim +
+                                    it.c * EPC) = y[i];
+        }
+      }
     }
   }
 }
