@@ -43,6 +43,12 @@ What it computes (sources are the pages this build follows):
   RMSNorm(head_dim = 128) applied before ``apply_rope``).  The pages print no eps
   for these two norms; callers pass it (the model's other RMSNorms use 1e-6).
 
+* ``linear`` -- the projections around the attention: Y = X W^T + b with
+  the nn.Linear weight layout W[N, K] (close reading, section 6: to_q, to_k,
+  to_v make the joint Q, K, V from the hidden states and to_out maps the
+  attention output back); in steps 2..N only the target tokens' rows are
+  projected (overview, card 6A).
+
 Inputs are arrays already cast to the GPU dtype (bf16 or fp32) by the seeded
 input module; every function promotes them to float64 first.
 
@@ -262,6 +268,20 @@ def attn_cached(q_t, k_t, v_t, pos_t, k_cache, v_cache, heads=None, rows=None, b
             q_rot = rope(q_t[b, rows, h, :], pos_t[rows])
             out[bi, :, hi, :] = attention_head(q_rot, keys, vals, None)
     return out
+
+
+# ----------------------------------------------------------------------------
+# projections (Q/K/V in, attention output out)
+# ----------------------------------------------------------------------------
+
+def linear(x, w, bias=None):
+    """Y = X W^T (+ b) for ``x[..., K]``, ``w[N, K]``, ``bias[N]``; float64."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    y = x @ w.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)
+    return y
 
 
 # ----------------------------------------------------------------------------

@@ -290,11 +290,32 @@ def check_rms_norm_closed_forms(O):
     assert np.allclose(O.rms_norm(x, w, 1e-6), O.rms_norm(x, ones, 1e-6) * w, rtol=1e-15, atol=0)
 
 
+# ------------------------------------------------------------- projections --
+
+def check_linear_brute_force(O):
+    """Y[i, n] = sum_k X[i, k] W[n, k] + b[n], by explicit loops on a tiny case."""
+    rng = np.random.default_rng(13)
+    x, w, b = rng.standard_normal((3, 5)), rng.standard_normal((4, 5)), rng.standard_normal(4)
+    want = np.array([[sum(x[i, k] * w[n, k] for k in range(5)) + b[n] for n in range(4)] for i in range(3)])
+    assert np.max(np.abs(O.linear(x, w, b) - want)) < 1e-13
+    assert np.max(np.abs(O.linear(x, w) - (want - b))) < 1e-13
+
+
+def check_linear_special_cases(O):
+    """Identity weights reproduce X; zero input gives the bias; batched rows."""
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((2, 6, 8))
+    assert np.array_equal(O.linear(x, np.eye(8)), x)
+    b = rng.standard_normal(3)
+    assert np.array_equal(O.linear(np.zeros((4, 8)), rng.standard_normal((3, 8)), b), np.tile(b, (4, 1)))
+
+
 CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_frames,
           check_prompt_length_invariance, check_block_causal_rule, check_prefix_never_sees_target,
           check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
           check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
-          check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms]
+          check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms,
+          check_linear_brute_force, check_linear_special_cases]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
@@ -399,6 +420,16 @@ def _rms_no_weight(x, weight, eps):
     return OM.rms_norm(x, np.ones(128), eps)
 
 
+def _linear_untransposed(x, w, bias=None):
+    x, w = np.asarray(x, dtype=np.float64), np.asarray(w, dtype=np.float64)
+    y = x @ w.reshape(w.shape[1], w.shape[0]) if w.shape[0] != w.shape[1] else x @ w
+    return y if bias is None else y + bias
+
+
+def _linear_no_bias(x, w, bias=None):
+    return OM.linear(x, w)
+
+
 MUTANTS = {
     "rope_sign": dict(rope=_rope_sign_flipped),
     "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
@@ -410,6 +441,8 @@ MUTANTS = {
     "rms_sum_not_mean": dict(rms_norm=_rms_sum_not_mean),
     "rms_eps_outside_root": dict(rms_norm=_rms_eps_outside),
     "rms_weight_dropped": dict(rms_norm=_rms_no_weight),
+    "linear_weight_untransposed": dict(linear=_linear_untransposed),
+    "linear_bias_dropped": dict(linear=_linear_no_bias),
 }
 
 
