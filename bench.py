@@ -228,6 +228,46 @@ def pct(xs, q):
     return float(np.percentile(np.asarray(xs, dtype=np.float64), q))
 
 
+def time_projections(qi, args, M, D, flush, dev):
+    """tcgen05 projections of the target tokens of a cached step: the fused
+    Q/K/V projection (N = 3 D, three outputs) and the output projection
+    (N = D), bf16 with synthetic seeded weights; cuBLAS (torch.matmul) on the
+    same shapes for context.  L2 flushed before each rep."""
+    g = torch.Generator(device="cpu").manual_seed(11)
+    mk = lambda *shape, scale=1.0: (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16).to(dev)
+    x = mk(M, D)
+    w_qkv, b_qkv = mk(3 * D, D, scale=D ** -0.5), mk(3 * D, scale=0.1)
+    w_o, b_o = mk(D, D, scale=D ** -0.5), mk(D, scale=0.1)
+    ws = qi.new_workspace(256, dev)
+    outs = [torch.empty((M, D), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    y = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = max(3, min(args.steps, 20))
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        pairs = [(ev(), ev()) for _ in range(reps)]
+        for a, b in pairs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return pct([a.elapsed_time(b) for a, b in pairs], 50)
+
+    out = {"M": M, "hidden": D, "weights": "synthetic N(0, 1/hidden), bias N(0, 0.01)", "reps": reps}
+    for name, w, b, o, n_out in (("qkv", w_qkv, b_qkv, outs, 3), ("out", w_o, b_o, [y], 1)):
+        flops = 2.0 * M * w.shape[0] * D
+        ms = timed(lambda: qi.linear(x, w, b, n_out=n_out, out=o, workspace=ws))
+        ms_ref = timed(lambda: torch.addmm(b, x, w.t()))
+        out[name] = {"N": int(w.shape[0]), "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                     "cublas_tflops": flops / (ms_ref * 1e-3) / 1e12}
+    assert qi.workspace_status(ws) == 0
+    return out
+
+
 def time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops):
     """The workload's denoising loop for one layer: step 1 full (cache store)
     and steps 2..N cached on fresh target inputs, timed eagerly (one library
@@ -345,6 +385,9 @@ def run_ours(args, world, rank, local):
     full_ms, cached_ms = sum(full_each), sum(cached_each)
     assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
 
+    # ---- the projections of a cached step's target tokens (fused Q/K/V, output)
+    proj = time_projections(qi, args, B * T, H * 128, flush, dev)
+
     # ---- the denoising loop (1 full + N-1 cached steps), eager and as a CUDA graph
     loop = None
     if cfg.get("cached_steps", 0) > 1 and not args.qk_norm:
@@ -427,6 +470,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    line["projections"] = proj
     if loop is not None:
         line["loop"] = loop
     print(json.dumps(line), flush=True)

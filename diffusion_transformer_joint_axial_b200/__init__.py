@@ -7,11 +7,11 @@ binding: it marshals torch tensors into that ABI and nothing else.
 """
 
 from ._binding import (QI21Error, Segment, alloc_cache, attn_cached, attn_full, cached_workspace_size,
-                       full_workspace_size, launch_count, load_library, new_workspace, rope_positions,
+                       full_workspace_size, launch_count, linear, load_library, new_workspace, rope_positions,
                        selftest_exp2, selftest_wait_timeout, time_next_attention, workspace_status, HEAD_DIM,
                        LIB_PATH)
 from .steploop import DenoiseLoop
 
 __all__ = ["DenoiseLoop", "QI21Error", "Segment", "alloc_cache", "attn_cached", "attn_full", "cached_workspace_size",
-           "full_workspace_size", "launch_count", "load_library", "new_workspace", "rope_positions",
+           "full_workspace_size", "launch_count", "linear", "load_library", "new_workspace", "rope_positions",
            "selftest_exp2", "selftest_wait_timeout", "time_next_attention", "workspace_status", "HEAD_DIM", "LIB_PATH"]

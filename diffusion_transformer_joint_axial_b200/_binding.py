@@ -28,7 +28,7 @@ EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_f
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
             "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
-            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm")
+            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear")
 
 
 class QI21Error(RuntimeError):
@@ -71,6 +71,8 @@ def load_library(path=LIB_PATH):
                                         _vp, _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
     L.qi21_attn_cached_qknorm.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
+    L.qi21_linear.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, ctypes.POINTER(_vp), _i32, _vp, _sz, _vp]
+    L.qi21_linear.restype = _i32
     L.qi21_workspace_status.argtypes = [_vp, _vp]
     L.qi21_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
     L.qi21_status_string.argtypes = [_i32]
@@ -268,6 +270,44 @@ def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk
                                               _ptr(k_cache), _ptr(v_cache), _ptr(out), *norm,
                                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                                               _stream(dev)))
+    return out
+
+
+def linear(x, w, bias=None, n_out=1, out=None, workspace=None):
+    """Y = X W^T (+ b) on the tensor cores, bf16 with fp32 accumulation.
+
+    x: [..., K], w: [N, K] (nn.Linear layout), bias: [N] or None, all bf16 on
+    one CUDA device.  The N output columns are cut into ``n_out`` equal
+    segments; returns the list of ``n_out`` tensors [..., N / n_out] (or fills
+    ``out``, a list of such tensors).
+    """
+    L_ = _cuda_lib()
+    dev = x.device
+    K = x.shape[-1]
+    N = w.shape[0]
+    lead = tuple(x.shape[:-1])
+    M = 1
+    for d in lead:
+        M *= int(d)
+    _need(x, "x", lead + (K,), torch.bfloat16, dev)
+    _need(w, "w", (N, K), torch.bfloat16, dev)
+    if bias is not None:
+        _need(bias, "bias", (N,), torch.bfloat16, dev)
+    if n_out < 1 or N % n_out != 0:
+        raise QI21Error(QI21_ERR_INVALID_ARG, "N=%d does not split into %d segments" % (N, n_out))
+    seg = N // n_out
+    if out is None:
+        out = [torch.empty(lead + (seg,), dtype=torch.bfloat16, device=dev) for _ in range(n_out)]
+    if len(out) != n_out:
+        raise QI21Error(QI21_ERR_INVALID_ARG, "need %d output tensors" % n_out)
+    for i, o in enumerate(out):
+        _need(o, "out[%d]" % i, lead + (seg,), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(WORKSPACE_HEADER_BYTES, dev)
+    ptrs = (_vp * n_out)(*[o.data_ptr() for o in out])
+    with torch.cuda.device(dev):
+        _check(L_.qi21_linear(M, N, K, _ptr(x), _ptr(w), _ptr(bias), ptrs, n_out, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(dev)))
     return out
 
 

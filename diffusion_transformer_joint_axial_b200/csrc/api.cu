@@ -2,6 +2,7 @@
 // workspace carving, and the kernel sequence of each entry point.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdint.h>
 #include <string.h>
 
 #include "../../include/qi21.h"
@@ -349,6 +350,43 @@ qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, 
     return fail(QI21_ERR_INVALID_ARG, "norm_q and norm_k must be given");
   return attn_cached_impl(B, H, P, T, dt, q, k, v, pos_tgt, k_cache, v_cache, o, norm_q, norm_k, eps,
                           workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
+                        void* const* out, int32_t n_out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (M < 0 || N < 0 || K < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return fail(QI21_ERR_INVALID_ARG, "M, N, K must be in [0, 2^31)");
+  if (n_out < 1 || n_out > 4) return fail(QI21_ERR_INVALID_ARG, "n_out must be in [1, 4] (got %d)", n_out);
+  if (N % n_out != 0 || (N / n_out) % 8 != 0)
+    return fail(QI21_ERR_INVALID_ARG, "N / n_out must be a whole multiple of 8 (N=%lld, n_out=%d)",
+                (long long)N, n_out);
+  if (K % 8 != 0) return fail(QI21_ERR_INVALID_ARG, "K must be a multiple of 8 (got %lld)", (long long)K);
+  if (M == 0 || N == 0) return QI21_OK;
+  if (K == 0) return fail(QI21_ERR_INVALID_ARG, "K must be >= 8 when M and N are not 0");
+  QI21_TRY(check_ptr(x, "x"));
+  QI21_TRY(check_ptr(w, "w"));
+  if (bias != nullptr) QI21_TRY(check_ptr(bias, "bias"));
+  if (out == nullptr) return fail(QI21_ERR_INVALID_ARG, "out is NULL");
+  for (int i = 0; i < n_out; ++i) QI21_TRY(check_ptr(out[i], "out[i]"));
+  QI21_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < QI21_WORKSPACE_HEADER_BYTES)
+    return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %d bytes", workspace_bytes,
+                QI21_WORKSPACE_HEADER_BYTES);
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.x = x;
+  a.w = w;
+  a.bias = bias;
+  for (int i = 0; i < n_out; ++i) a.out[i] = out[i];
+  a.n_out = n_out;
+  a.status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = launch_gemm_tc(a, static_cast<cudaStream_t>(stream), sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "linear launch");
+  return QI21_OK;
 }
 
 qi21_status qi21_workspace_status(void* workspace, void* stream) {

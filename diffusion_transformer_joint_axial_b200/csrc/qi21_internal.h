@@ -93,6 +93,20 @@ struct AttnArgs {
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);
 
+// ------------------------------------------------------------ linear layer
+// Y = X W^T (+ b): X [M, K], W [N, K], b [N] or null, all bf16; the N output
+// columns go to n_out equal segments out[i] = [M, N / n_out] (row-major).
+struct GemmArgs {
+  int64_t M, N, K;
+  const void* x;
+  const void* w;
+  const void* bias;
+  void* out[4];
+  int32_t n_out;
+  uint32_t* status;  // workspace header status word
+};
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);
+
 // --------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t stream);

@@ -182,6 +182,34 @@ qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, 
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qi21_linear -- the projections around the attention, on the tensor cores:
+ *     Y = X W^T (+ b)
+ * with X [M, K], W [N, K] (the nn.Linear weight layout: K contiguous) and b
+ * [N], all bf16, accumulated in fp32 and rounded once to bf16.  The joint
+ * attention's Q, K and V come from such projections of the hidden states and
+ * its output goes through one (close reading section 6: to_q / to_k / to_v,
+ * to_out); in steps 2..N only the target tokens' rows need projecting
+ * (overview card 6A), which is M = B * T here.  The N output columns are cut
+ * into n_out equal segments, segment i written to out[i] as a row-major
+ * [M, N / n_out] tensor: with W = [W_q; W_k; W_v] and n_out = 3 one launch
+ * leaves Q, K and V in the [B, T, H, 128] layout qi21_attn_* read.
+ *
+ *   M, N, K     sizes (>= 0; K a multiple of 8 and >= 8 unless M or N is 0).
+ *   x, w        device bf16 [M, K], [N, K], 16-byte aligned, read.
+ *   bias        device bf16 [N] (16-byte aligned) or NULL.
+ *   out         HOST array of n_out (1..4) device pointers, each 16-byte
+ *               aligned, [M, N / n_out] bf16 written; N / n_out must be a
+ *               multiple of 8.
+ *   workspace   device scratch of at least QI21_WORKSPACE_HEADER_BYTES (its
+ *               status header, as for qi21_attn_full).
+ * Returns QI21_ERR_INVALID_ARG for bad sizes, pointers or alignment before
+ * enqueuing anything.
+ */
+qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                        const void* bias, void* const* out, int32_t n_out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * qi21_attn_cached_noalloc -- the cached step of qi21_attn_cached for callers
  * that may not allocate device memory (plugin hosts that only hand over a
  * stream and tensors, servers that reserve all memory at start-up, loops where

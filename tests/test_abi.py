@@ -147,6 +147,27 @@ def test_qknorm_rejects(lib):
         assert "eps" in lib.qi21_last_error().decode()
 
 
+def test_linear_rejects(lib):
+    p = ctypes.c_void_p
+    outs = (p * 4)(16, 16, 16, 16)
+    lin = lambda M=64, N=96, K=64, x=16, w=16, b=None, out=outs, n=1, ws=256, wsb=256: lib.qi21_linear(
+        M, N, K, p(x) if x else None, p(w) if w else None, p(b) if b else None, out, n,
+        p(ws) if ws else None, wsb, None)
+    bad = qb.QI21_ERR_INVALID_ARG
+    assert lin(n=0) == bad and lin(n=5) == bad          # segment count
+    assert lin(N=96, n=5) == bad                         # N not divisible
+    assert lin(N=36, n=3) == bad                         # segment not a multiple of 8
+    assert lin(K=60) == bad                              # K not a multiple of 8
+    assert lin(K=0) == bad
+    assert lin(M=-1) == bad
+    assert lin(x=None) == bad and lin(w=24) == bad       # NULL / misaligned operand
+    assert lin(b=40) == bad                              # misaligned bias
+    assert lin(out=None) == bad
+    assert lin(out=(p * 4)(16, 20, 16, 16), N=96, n=2) == bad  # misaligned second output
+    assert lin(wsb=100) == bad                           # workspace smaller than its header
+    assert lin(M=0, x=None, w=None, ws=None) == qb.QI21_OK  # nothing to do
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.qi21_selftest_wait_timeout(ctypes.c_void_p(256), 0, None) == qb.QI21_ERR_INVALID_ARG
 
