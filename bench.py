@@ -300,6 +300,39 @@ def time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops):
            "tflops_graph": flops / (g * 1e-3) / 1e12}
     del loop
     torch.cuda.empty_cache()
+
+    # the same loop as attention sublayers: projections of each step's tokens
+    # (step 1 all L, later steps the T target tokens) around the attention
+    B, H = cfg["B"], cfg["H"]
+    L, P, T = W.sizes(name)
+    D = H * 128
+    layer = qi.DenoiseLoop(cfg["segments"], B, H, n, torch.bfloat16, dev, projections=True)
+    g = torch.Generator(device="cpu").manual_seed(12)
+    rnd = lambda *shape, scale=1.0: (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16)
+    layer.load_layer(rnd(B, L, D), [rnd(B, T, D) for _ in range(n - 1)], rnd(3 * D, D, scale=D ** -0.5),
+                     rnd(3 * D, scale=0.1), rnd(D, D, scale=D ** -0.5), rnd(D, scale=0.1))
+    layer.capture()
+    for _ in range(2):
+        layer.replay()
+    ev = [(mk(), mk()) for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        layer.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    layer.check()
+    lt = [a.elapsed_time(b) for a, b in ev]
+    proj_flops = 2.0 * 4 * D * D * B * (L + (n - 1) * T)  # Q/K/V (3 D x D) + output (D x D)
+    gl = pct(lt, 50)
+    out["layer"] = {"what": "attention sublayer: fused Q/K/V projection -> attention -> output projection, "
+                            "synthetic weights; step 1 projects all %d tokens, steps 2..%d the %d target "
+                            "tokens" % (L, n, T),
+                    "graph_ms_median": gl, "graph_ms_p95": pct(lt, 95),
+                    "tflops_graph": (flops + proj_flops) / (gl * 1e-3) / 1e12,
+                    "projection_tflop": proj_flops / 1e12}
+    del layer
+    torch.cuda.empty_cache()
     return out
 
 
