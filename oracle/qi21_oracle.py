@@ -20,6 +20,12 @@ What it computes (sources are the pages this build follows):
   overview, card 3C (text reads only what precedes it, tokens of one image see
   each other both ways) and the learning goals (the Prefix never attends the
   target); the target is appended last (card 2A).
+* ``positions_original`` -- the earlier Qwen-Image model's table, a second
+  workload for the same attention: images are numbered as above, text tokens
+  continue after the images, f = h = w = max_vid_index + running text index
+  with max_vid_index the largest max(H//2, W//2) over the images, and there
+  is no mask (close reading, section 7.2: ``txt_freqs`` taken from
+  ``max_vid_index`` on; section 6: ``is_causal=False``, text sees the images).
 * ``rope_angles`` / ``rope`` -- axial rotary embedding: head_dim 128 split
   into bands (16, 56, 56) for (frame, height, width) (3A, section 1); per axis
   the angle of pair j is pos * theta^(-2j/d_axis) with theta = 10000 (close
@@ -117,6 +123,35 @@ def allowed_matrix(kv_end, n_keys):
     """Dense boolean mask: allowed[i, j] = j < kv_end[i]."""
     kv_end = np.asarray(kv_end, dtype=np.int64)
     return np.arange(n_keys)[None, :] < kv_end[:, None]
+
+
+def positions_original(segments):
+    """The earlier model's position table and (absent) mask.
+
+    Image tokens get the same (frame, h, w) as in ``positions`` (close
+    reading, section 7.3: negative table tail then positive table head, frame
+    = the image's index).  Text tokens get f = h = w = max_vid_index + j for
+    the j-th text token, where max_vid_index = max over the images of
+    max(H//2, W//2) (section 7.2, ``scale_rope``): text continues beyond the
+    images.  No mask: every token sees all L keys (section 6).
+    """
+    pos, _ = positions(segments)
+    max_vid_index = 0
+    for seg in segments:
+        if seg["kind"] == "image":
+            max_vid_index = max(max_vid_index, int(seg["H"]) // 2, int(seg["W"]) // 2)
+    start = 0
+    text_counter = 0
+    for seg in segments:
+        n = int(seg["n"]) if seg["kind"] == "text" else int(seg["H"]) * int(seg["W"])
+        if seg["kind"] == "text":
+            for t in range(n):
+                v = max_vid_index + text_counter
+                pos[start + t] = (v, v, v)
+                text_counter += 1
+        start += n
+    kv_end = np.full(start, start, dtype=np.int32)
+    return pos, kv_end
 
 
 # ----------------------------------------------------------------------------

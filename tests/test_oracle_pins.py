@@ -290,6 +290,24 @@ def check_rms_norm_closed_forms(O):
     assert np.allclose(O.rms_norm(x, w, 1e-6), O.rms_norm(x, ones, 1e-6) * w, rtol=1e-15, atol=0)
 
 
+# ------------------------------------------------- earlier model's positions --
+
+def check_original_text_offset(O):
+    """Close reading 7.2: the earlier model's text continues after the images,
+    from max over images of max(H//2, W//2), +1 per text token on all axes;
+    images keep the centred grid of 7.3; no mask (section 6)."""
+    segs = [W.text(3), W.image(4, 6, 0), W.image(10, 2, 1)]  # max(2, 3, 5, 1) = 5
+    pos, kv = O.positions_original(segs)
+    assert [tuple(int(x) for x in p) for p in pos[:3]] == [(5, 5, 5), (6, 6, 6), (7, 7, 7)]
+    assert np.array_equal(pos[3:], O.positions(segs)[0][3:])
+    assert np.all(np.asarray(kv) == len(pos))
+    img = np.asarray(pos[3:])
+    assert pos[0][1] > img[:, 1].max() and pos[0][2] > img[:, 2].max()
+    # the earlier model's edit layout: [text | target 64x64 | reference 64x64] -> text from 32
+    pos2, _ = O.positions_original([W.text(2), W.image(64, 64, 0), W.image(64, 64, 1)])
+    assert [tuple(int(x) for x in p) for p in pos2[:2]] == [(32, 32, 32), (33, 33, 33)]
+
+
 # ------------------------------------------------------------- projections --
 
 def check_linear_brute_force(O):
@@ -315,7 +333,7 @@ CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_f
           check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
           check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
           check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms,
-          check_linear_brute_force, check_linear_special_cases]
+          check_linear_brute_force, check_linear_special_cases, check_original_text_offset]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
@@ -430,6 +448,25 @@ def _linear_no_bias(x, w, bias=None):
     return OM.linear(x, w)
 
 
+def _original_offset_unhalved(segments):
+    """Text offset max(H, W) (the earlier model's scale_rope=False branch)."""
+    pos, kv = OM.positions_original(segments)
+    imgs = [s for s in segments if s["kind"] == "image"]
+    shift = max(max(s["H"], s["W"]) for s in imgs) - max(max(s["H"] // 2, s["W"] // 2) for s in imgs)
+    start = 0
+    for seg in segments:
+        n = W.seg_tokens(seg)
+        if seg["kind"] == "text":
+            pos[start:start + n] += shift
+        start += n
+    return pos, kv
+
+
+def _original_from_zero(segments):
+    _, kv = OM.positions_original(segments)
+    return OM.positions(segments)[0], kv
+
+
 MUTANTS = {
     "rope_sign": dict(rope=_rope_sign_flipped),
     "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
@@ -443,6 +480,8 @@ MUTANTS = {
     "rms_weight_dropped": dict(rms_norm=_rms_no_weight),
     "linear_weight_untransposed": dict(linear=_linear_untransposed),
     "linear_bias_dropped": dict(linear=_linear_no_bias),
+    "original_offset_unhalved": dict(positions_original=_original_offset_unhalved),
+    "original_text_from_zero": dict(positions_original=_original_from_zero),
 }
 
 
