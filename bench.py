@@ -57,9 +57,12 @@ def ncu_traffic(name):
 # ------------------------------------------------------------------ helpers --
 
 def step_flops(name):
-    """Algorithmic FLOPs of one step: full step + one cached step, all heads."""
+    """Algorithmic FLOPs of one step: full step + one cached step, all heads
+    (the earlier model's workload: one unmasked full step, no cached step)."""
     cfg = W.WORKLOADS[name]
     L, P, T = W.sizes(name)
+    if cfg.get("original"):
+        return 4.0 * 128 * L * L * cfg["B"] * cfg["H"], 0.0
     # allowed pairs of the full step: sum over rows of their visibility bound
     # (the segment layout fixes it: text token i sees i + 1 keys, an image
     # token sees everything up to the end of its image)
@@ -97,7 +100,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             # nvidia-smi takes a moment to start: wait for its first sample
             # (taken before the timed region, not counted) so that sampling
@@ -175,14 +178,16 @@ def oracle_sample(name, budget_s):
     L, P, T = W.sizes(name)
     q, k, v = W.draw_qkv(1, L, 1, cfg["seed"], cfg["dtype"])
     qf, kf, vf = W.as_f64(q), W.as_f64(k), W.as_f64(v)
-    pos, kv_end = O.positions(cfg["segments"])
+    orig = cfg.get("original", False)
+    pos, kv_end = (O.positions_original if orig else O.positions)(cfg["segments"])
     full1, cached1 = (x / (cfg["B"] * cfg["H"]) for x in step_flops(name))
     flops, heads = 0.0, 0
     t0 = time.perf_counter()
     while True:
         O.attn_full(qf, kf, vf, pos, kv_end)
-        kc, vc = O.prefix_cache(kf, vf, pos, P)
-        O.attn_cached(qf[:, P:], kf[:, P:], vf[:, P:], pos[P:], kc, vc)
+        if not orig:
+            kc, vc = O.prefix_cache(kf, vf, pos, P)
+            O.attn_cached(qf[:, P:], kf[:, P:], vf[:, P:], pos[P:], kc, vc)
         flops += full1 + cached1
         heads += 1
         dt = time.perf_counter() - t0
@@ -209,8 +214,9 @@ def run_reference(args, world, rank):
         f, s, h = oracle_sample(name, 0.0)
         tot_f, tot_s, heads = tot_f + f, tot_s + s, heads + h
     value = tot_f / tot_s / 1e12
-    sample = "%d head(s) of the %s full step + one cached step per bench step (float64 oracle, %s)" % (
-        heads // max(1, args.steps), name, W.DESCRIPTIONS[name])
+    sample = "%d head(s) of the %s full step%s per bench step (float64 oracle, %s)" % (
+        heads // max(1, args.steps), name, "" if cfg.get("original") else " + one cached step",
+        W.DESCRIPTIONS[name])
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -347,17 +353,20 @@ def run_ours(args, world, rank, local):
     L, P, T = W.sizes(name)
     segs = cfg["segments"]
     dt = torch.bfloat16
+    # the earlier model's workload: positions with text after the images, one
+    # unmasked full step, nothing cached (its text attends the target)
+    orig = cfg.get("original", False)
 
     # inputs (host, pinned) and device-resident copies
     q, k, v = W.full_inputs(name)
-    qt, kt, vt = W.cached_inputs(name, 2)
-    host = [x.pin_memory() for x in (q, k, v, qt, kt, vt)]
-    dq, dk, dv, dqt, dkt, dvt = (x.to(dev) for x in host)
-    kc, vc = qi.alloc_cache(B, H, P, dt, dev)
+    host = [x.pin_memory() for x in ((q, k, v) if orig else (q, k, v) + tuple(W.cached_inputs(name, 2)))]
+    dq, dk, dv = (x.to(dev) for x in host[:3])
+    dqt, dkt, dvt = (None, None, None) if orig else (x.to(dev) for x in host[3:])
+    kc, vc = (None, None) if orig else qi.alloc_cache(B, H, P, dt, dev)
     o_full = torch.empty_like(dq)
-    o_c = torch.empty_like(dqt)
+    o_c = None if orig else torch.empty_like(dqt)
     ws_f = qi.new_workspace(qi.full_workspace_size(B, H, L, P, dt), dev)
-    ws_c = qi.new_workspace(qi.cached_workspace_size(B, H, P, T, dt), dev)
+    ws_c = qi.new_workspace(256 if orig else qi.cached_workspace_size(B, H, P, T, dt), dev)
     pos = torch.empty((L, 3), dtype=torch.int32, device=dev)
     kv_end = torch.empty((L,), dtype=torch.int32, device=dev)
     assert pos[P:].data_ptr() % 16 == 0, "target rows of the position table must be 16-byte aligned"
@@ -376,13 +385,20 @@ def run_ours(args, world, rank, local):
     else:
         full_fn, cached_fn = lib.qi21_attn_full, lib.qi21_attn_cached
 
+    positions_fn = lib.qi21_rope_positions_original if orig else lib.qi21_rope_positions
+
     def one_step(ev=None, qq=dq, kk=dk, vv=dv, qqt=dqt, kkt=dkt, vvt=dvt):
-        lib.qi21_rope_positions(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
+        positions_fn(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
         if ev is not None:
             qi.time_next_attention(ev[0], ev[1])
-        st = full_fn(B, H, L, P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
+        st = full_fn(B, H, L, 0 if orig else P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
                      P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
         assert st == 0, lib.qi21_last_error()
+        if orig:
+            if ev is not None:  # no cached step: an empty interval keeps the bookkeeping
+                ev[2].record(stream)
+                ev[3].record(stream)
+            return
         if ev is not None:
             qi.time_next_attention(ev[2], ev[3])
         st = cached_fn(B, H, P, T, 0, P_(qqt), P_(kkt), P_(vvt), P_(pos[P:]), P_(kc), P_(vc),
@@ -428,9 +444,9 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the C ABI with host buffers (copies timed)
     h2d = sum(x.numel() * x.element_size() for x in host)
-    d2h = (o_full.numel() + o_c.numel()) * 2
-    out_h = [torch.empty(o_full.shape, dtype=dt, pin_memory=True),
-             torch.empty(o_c.shape, dtype=dt, pin_memory=True)]
+    outs_d = [o_full] if orig else [o_full, o_c]
+    d2h = sum(o.numel() for o in outs_d) * 2
+    out_h = [torch.empty(o.shape, dtype=dt, pin_memory=True) for o in outs_d]
     e2e_steps = max(3, min(args.steps, 20))
     ee = [(mk(), mk()) for _ in range(e2e_steps)]
     barrier(world)
@@ -441,8 +457,8 @@ def run_ours(args, world, rank, local):
         for d, h in zip((dq, dk, dv, dqt, dkt, dvt), host):
             d.copy_(h, non_blocking=True)
         one_step()
-        out_h[0].copy_(o_full, non_blocking=True)
-        out_h[1].copy_(o_c, non_blocking=True)
+        for hh, dd in zip(out_h, outs_d):
+            hh.copy_(dd, non_blocking=True)
         ee[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
@@ -469,30 +485,33 @@ def run_ours(args, world, rank, local):
     att_ms = full_ms + cached_ms
     achieved = (full_flops + cached_flops) * args.steps / (att_ms * 1e-3) / 1e12
     full_tf = full_flops * args.steps / (full_ms * 1e-3) / 1e12
-    cached_tf = cached_flops * args.steps / (cached_ms * 1e-3) / 1e12
+    cached_tf = cached_flops * args.steps / (cached_ms * 1e-3) / 1e12 if cached_flops else None
 
     budget = 0.0 if args.no_cpu_baseline else args.cpu_budget
     cpu = None
     if budget > 0:
         f, s, heads = oracle_sample(name, budget)
         cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": "%d of %d (batch, head) pairs of the %s step (full + one cached), float64 "
-                         "NumPy oracle, %.1f s" % (heads, B * H, name, s)}
+               "sample": "%d of %d (batch, head) pairs of the %s step (%s), float64 "
+                         "NumPy oracle, %.1f s" % (heads, B * H, name,
+                                                   "one unmasked full step" if orig else "full + one cached",
+                                                   s)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": W.DESCRIPTIONS[name], "B": B, "H": H, "L": L, "P": P, "T": T,
-                   "step": "positions + full block-causal step with cache store + one cached step"
+                   "step": ("positions (text after the images) + one unmasked full step" if orig else
+                            "positions + full block-causal step with cache store + one cached step")
                            + (", QK-RMSNorm fused (synthetic weights)" if args.qk_norm else ""),
                    "qk_norm": bool(args.qk_norm),
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "dp%d (independent requests per GPU)" % world},
         "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps,
                       "ms_median": pct(full_each, 50), "ms_p95": pct(full_each, 95)},
-        "cached_step": {"tflops": cached_tf, "frac_of_peak": cached_tf / peak,
-                        "ms": cached_ms / args.steps, "ms_median": pct(cached_each, 50),
-                        "ms_p95": pct(cached_each, 95)},
+        "cached_step": None if orig else {
+            "tflops": cached_tf, "frac_of_peak": cached_tf / peak, "ms": cached_ms / args.steps,
+            "ms_median": pct(cached_each, 50), "ms_p95": pct(cached_each, 95)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": ncu_traffic(name), "traffic_unit": "bytes/launch",
                      "kernel": "qi21::tc::attn_tc_kernel (full + cached launches)",

@@ -28,7 +28,7 @@ EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_f
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
             "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
-            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear")
+            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear", "qi21_rope_positions_original")
 
 
 class QI21Error(RuntimeError):
@@ -59,6 +59,8 @@ def load_library(path=LIB_PATH):
                         "libqi21.so is not built (python -m diffusion_transformer_joint_axial_b200.build)")
     L = ctypes.CDLL(path)
     L.qi21_rope_positions.argtypes = [ctypes.POINTER(Segment), _i32, _i64, _vp, _vp, _vp]
+    L.qi21_rope_positions_original.argtypes = [ctypes.POINTER(Segment), _i32, _i64, _vp, _vp, _vp]
+    L.qi21_rope_positions_original.restype = _i32
     L.qi21_attn_full_workspace_size.argtypes = [_i32, _i32, _i64, _i64, _i32]
     L.qi21_attn_full_workspace_size.restype = _sz
     L.qi21_attn_full.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -147,8 +149,11 @@ def to_segments(segments):
     return arr
 
 
-def rope_positions(segments, device="cuda", with_kv_end=True):
-    """Position table ``pos[L, 3]`` (int32) and ``kv_end[L]`` on ``device``."""
+def rope_positions(segments, device="cuda", with_kv_end=True, original=False):
+    """Position table ``pos[L, 3]`` (int32) and ``kv_end[L]`` on ``device``.
+
+    ``original=True`` builds the earlier model's table (text after the
+    images, no mask; ``qi21_rope_positions_original``)."""
     L_ = _cuda_lib()
     device = torch.device(device)
     if device.index is None:
@@ -158,7 +163,8 @@ def rope_positions(segments, device="cuda", with_kv_end=True):
     pos = torch.empty((n, 3), dtype=torch.int32, device=device)
     kv_end = torch.empty((n,), dtype=torch.int32, device=device) if with_kv_end else None
     with torch.cuda.device(device):
-        _check(L_.qi21_rope_positions(segs, len(segments), n, _ptr(pos), _ptr(kv_end), _stream(device)))
+        fn = L_.qi21_rope_positions_original if original else L_.qi21_rope_positions
+        _check(fn(segs, len(segments), n, _ptr(pos), _ptr(kv_end), _stream(device)))
     return pos, kv_end
 
 

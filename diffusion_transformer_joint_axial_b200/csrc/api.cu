@@ -107,8 +107,11 @@ using namespace qi21;
 
 extern "C" {
 
-qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_t L, int32_t* pos,
-                                int32_t* kv_end, void* stream) {
+// Position table and visibility bound.  original = the earlier model: text
+// positions start after the images (max over images of max(H//2, W//2)) and
+// there is no mask.
+static qi21_status rope_positions_impl(const qi21_segment* segs, int32_t n_segs, int64_t L, int32_t* pos,
+                                       int32_t* kv_end, bool original, void* stream) {
   if (n_segs == 0 && L == 0) return QI21_OK;
   if (segs == nullptr) return fail(QI21_ERR_INVALID_ARG, "segs is NULL");
   if (n_segs < 1 || n_segs > QI21_MAX_SEGMENTS)
@@ -141,13 +144,33 @@ qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_
     if (start > INT32_MAX / 2) return fail(QI21_ERR_INVALID_ARG, "sequence too long");
   }
   if (start != L) return fail(QI21_ERR_INVALID_ARG, "segments hold %lld tokens, L = %lld", (long long)start, (long long)L);
+  if (original) {
+    int32_t max_vid_index = 0;
+    for (int i = 0; i < n_segs; ++i)
+      if (segs[i].kind == QI21_SEG_IMAGE) {
+        max_vid_index = segs[i].H / 2 > max_vid_index ? segs[i].H / 2 : max_vid_index;
+        max_vid_index = segs[i].W / 2 > max_vid_index ? segs[i].W / 2 : max_vid_index;
+      }
+    for (int i = 0; i < n_segs; ++i) p.segs[i].text_base += max_vid_index;
+  }
   p.n_segs = n_segs;
   p.L = L;
   p.pos = pos;
   p.kv_end = kv_end;
+  p.all_visible = original ? 1 : 0;
   cudaError_t e = launch_positions(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "positions launch");
   return QI21_OK;
+}
+
+qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_t L, int32_t* pos,
+                                int32_t* kv_end, void* stream) {
+  return rope_positions_impl(segs, n_segs, L, pos, kv_end, false, stream);
+}
+
+qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_segs, int64_t L, int32_t* pos,
+                                         int32_t* kv_end, void* stream) {
+  return rope_positions_impl(segs, n_segs, L, pos, kv_end, true, stream);
 }
 
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt) {

@@ -10,9 +10,11 @@ namespace qi21 {
 // ============================================================== positions ==
 // One thread per token.  "3A - 3D Axial RoPE (16, 56, 56) & Zero-Centered
 // Grid", section 1: text advances (f, h, w) together by +1 (counting text
-// tokens only, from 0); an image freezes f and centres its row-major grid,
-// h = r - (H - H//2), w = c - (W - W//2).  Visibility bound (overview card 3C):
-// text token i sees [0, i]; an image token sees up to the end of its image.
+// tokens only, from the segment's text_base); an image freezes f and centres
+// its row-major grid, h = r - (H - H//2), w = c - (W - W//2).  Visibility
+// bound (overview card 3C): text token i sees [0, i]; an image token sees up
+// to the end of its image; with all_visible (the earlier model, no mask)
+// every token sees all L keys.
 __global__ void positions_kernel(const __grid_constant__ PositionsParams p) {
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= p.L) return;
@@ -36,6 +38,7 @@ __global__ void positions_kernel(const __grid_constant__ PositionsParams p) {
     w = c - (s.W - s.W / 2);
     end = s.start + s.H * s.W;
   }
+  if (p.all_visible) end = static_cast<int32_t>(p.L);
   p.pos[3 * i + 0] = f;
   p.pos[3 * i + 1] = h;
   p.pos[3 * i + 2] = w;

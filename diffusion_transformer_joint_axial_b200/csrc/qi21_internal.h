@@ -28,7 +28,7 @@ struct WsHeader {
 struct SegDev {
   int32_t kind, n, H, W, frame;
   int32_t start;      // first token of the segment
-  int32_t text_base;  // text tokens before the segment
+  int32_t text_base;  // position of the segment's first text token
 };
 constexpr int kMaxSegments = 128;
 struct PositionsParams {
@@ -37,6 +37,7 @@ struct PositionsParams {
   int64_t L;
   int32_t* pos;
   int32_t* kv_end;
+  int32_t all_visible;  // 1: no mask, every token sees all L keys
 };
 cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream);
 

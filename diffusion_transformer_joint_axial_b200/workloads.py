@@ -46,6 +46,11 @@ WORKLOADS = {
                    + [image(64, 64, 0)]),
     "hires": dict(dtype="bf16", B=2, H=24, seed=4,
                   segments=[text(512), image(64, 64, 1), image(128, 128, 0)]),
+    # the earlier Qwen-Image model's edit layout: [text | target | reference],
+    # text positions after the images, no mask (full step only: nothing is
+    # cacheable when the text attends the target)
+    "orig": dict(dtype="bf16", B=1, H=24, seed=5, original=True,
+                 segments=[text(256), image(64, 64, 0), image(64, 64, 1)]),
 }
 
 DESCRIPTIONS = {
@@ -54,6 +59,7 @@ DESCRIPTIONS = {
     "edit3": "edit with 3 references: B=1, 24 heads, text 512 + 3x(64x64) + target 64x64 (L=16896)",
     "maxref": "max-reference 8-step loop: B=1, 24 heads, text 1024 + 10x(48x48) + target 64x64 (L=28160)",
     "hires": "high-res 2048^2: B=2, 24 heads, text 512 + ref 64x64 + target 128x128 (L=20992)",
+    "orig": "earlier-model edit: B=1, 24 heads, text 256 + target 64x64 + ref 64x64, no mask (L=8448)",
 }
 
 

@@ -88,6 +88,20 @@ typedef struct {
 qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_t L,
                                 int32_t* pos, int32_t* kv_end, void* stream);
 
+/*
+ * qi21_rope_positions_original -- the same table for the earlier Qwen-Image
+ * model, a second workload for the attention with the mask off.  Images are
+ * numbered exactly as above (close reading section 7.3); text tokens take
+ * f = h = w = max_vid_index + (text tokens before them), where max_vid_index
+ * is the largest max(H//2, W//2) over the image segments (section 7.2: the
+ * text frequencies start at max_vid_index); kv_end[i] = L for every token (no
+ * mask; section 6: is_causal=False).  That model orders its sequence
+ * [text | target | references]; the segment order is the caller's.  Same
+ * arguments, errors and layout as qi21_rope_positions.
+ */
+qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_segs, int64_t L,
+                                         int32_t* pos, int32_t* kv_end, void* stream);
+
 /* Workspace bytes qi21_attn_full needs for these sizes (header included). */
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt);
 

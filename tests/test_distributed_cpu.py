@@ -51,12 +51,13 @@ def test_single_rank_is_identity():
     assert bench.sum_over_ranks(3.0, 1, None) == 3.0
 
 
-@pytest.mark.parametrize("name", ["tiny", "t2i", "edit3", "maxref", "hires"])
+@pytest.mark.parametrize("name", ["tiny", "t2i", "edit3", "maxref", "hires", "orig"])
 def test_bench_flops_match_oracle_pair_count(name):
     cfg = W.WORKLOADS[name]
     L, P, T = W.sizes(name)
-    _, kv_end = O.positions(cfg["segments"])
+    orig = cfg.get("original", False)
+    _, kv_end = (O.positions_original if orig else O.positions)(cfg["segments"])
     full, cached = bench.step_flops(name)
     bh = cfg["B"] * cfg["H"]
     assert full == 4 * 128 * O.allowed_pairs(kv_end) * bh
-    assert cached == 4 * 128 * T * (P + T) * bh
+    assert cached == (0 if orig else 4 * 128 * T * (P + T) * bh)
