@@ -120,6 +120,50 @@ def qk_norm_weights(seed=7):
                  for _ in range(2))
 
 
+# The denoising loop's synthetic model (the pages publish no trained
+# weights).  Widths: D = 128 * heads, a 3x wider SwiGLU hidden layer, C latent
+# channels.  Weights N(0, 1/fan_in), norm weights 1 + 0.1 N(0, 1), biases
+# 0.02 N(0, 1), the per-step embedding biases (the target's conditioning)
+# 0.5 N(0, 1); latents and Prefix hidden states N(0, 1).  Sigmas
+# linspace(1, 1/S, S) followed by 0.
+
+
+def denoise_sigmas(steps):
+    return [1.0 - i * (1.0 - 1.0 / steps) / max(1, steps - 1) for i in range(steps)] + [0.0]
+
+
+def denoise_model(heads, channels, blocks, steps, seed, dtype="bf16"):
+    """(params, draw) for the denoising loop: ``params`` as the oracle's
+    ``denoise`` takes them (CPU torch tensors of ``dtype``); ``draw(B, P, T,
+    seed)`` gives (x0 [B, T, C], prefix_h [B, P, D])."""
+    rng = np.random.default_rng(seed)
+    D, F, C = heads * HEAD_DIM, 3 * heads * HEAD_DIM, channels
+
+    def t(a):
+        x = torch.from_numpy(np.asarray(a, dtype=np.float32))
+        return x.to(torch.bfloat16) if dtype == "bf16" else x
+
+    def w(n, k):
+        return t(rng.standard_normal((n, k)) / np.sqrt(k))
+
+    def b(n, scale=0.02):
+        return t(scale * rng.standard_normal(n))
+
+    blk = []
+    for _ in range(blocks):
+        blk.append(dict(norm1=t(1 + 0.1 * rng.standard_normal(D)), w_qkv=w(3 * D, D), b_qkv=b(3 * D),
+                        w_o=w(D, D), b_o=b(D), norm2=t(1 + 0.1 * rng.standard_normal(D)),
+                        w_gu=w(2 * F, D), b_gu=b(2 * F), w_down=w(D, F), b_down=b(D)))
+    params = dict(w_in=w(D, C), b_in=t(0.5 * rng.standard_normal((steps, D))), blocks=blk,
+                  norm_out=t(1 + 0.1 * rng.standard_normal(D)), w_v=w(C, D), b_v=b(C))
+
+    def draw(B, P, T, seed2):
+        r = np.random.default_rng(seed2)
+        return t(r.standard_normal((B, T, C))), t(r.standard_normal((B, P, D)))
+
+    return params, draw
+
+
 def as_f64(t):
     """float64 numpy copy of a (CPU) torch tensor, for the oracle."""
     return t.detach().to("cpu").to(torch.float64).numpy()

@@ -55,6 +55,17 @@ What it computes (sources are the pages this build follows):
   attention output back); in steps 2..N only the target tokens' rows are
   projected (overview, card 6A).
 
+* ``silu`` / ``denoise`` -- the denoising loop around the attention: each
+  step embeds the target latents, runs the stack of blocks (RMSNorm ->
+  attention -> residual, RMSNorm -> SwiGLU with a 3x wider hidden layer ->
+  residual; overview cards 4A and 5A), maps the target tokens to a velocity
+  and takes the Euler step x <- x + (sigma_next - sigma) v (card 6B and the
+  learning goals).  The Prefix tokens take no step-dependent input, so in
+  the cached form step 1 runs every token and stores each block's Prefix
+  K/V, and later steps run the target tokens only (card 6A); the full form
+  recomputes everything at every step.  The pages' lab finds both equal to
+  about 1e-16.
+
 Inputs are arrays already cast to the GPU dtype (bf16 or fp32) by the seeded
 input module; every function promotes them to float64 first.
 
@@ -200,10 +211,11 @@ def rope(x, pos):
 # ----------------------------------------------------------------------------
 
 def rms_norm(x, weight, eps):
-    """RMSNorm over the last axis (head_dim 128): x / sqrt(mean(x^2) + eps) * weight."""
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * weight (head_dim
+    128 for the QK norm, the model width for the block norms)."""
     x = np.asarray(x, dtype=np.float64)
     weight = np.asarray(weight, dtype=np.float64)
-    assert x.shape[-1] == HEAD_DIM and weight.shape == (HEAD_DIM,)
+    assert weight.shape == (x.shape[-1],)
     ms = np.mean(x * x, axis=-1, keepdims=True)
     return x / np.sqrt(ms + eps) * weight
 
@@ -317,6 +329,76 @@ def linear(x, w, bias=None):
     if bias is not None:
         y = y + np.asarray(bias, dtype=np.float64)
     return y
+
+
+# ----------------------------------------------------------------------------
+# the denoising loop: blocks of attention + SwiGLU, Euler steps
+# ----------------------------------------------------------------------------
+
+def silu(x):
+    """x * sigmoid(x)."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def _split(y, parts):
+    n = y.shape[-1] // parts
+    return [y[..., i * n:(i + 1) * n] for i in range(parts)]
+
+
+def _block_attention(h, blk, eps, attend):
+    """h + (attend(q, k, v) W_o^T + b_o) with q, k, v from RMSNorm(h)."""
+    B, L, D = h.shape
+    a = rms_norm(h, blk["norm1"], eps)
+    q, k, v = (t.reshape(B, L, D // HEAD_DIM, HEAD_DIM) for t in _split(linear(a, blk["w_qkv"], blk["b_qkv"]), 3))
+    o = attend(q, k, v)
+    return h + linear(o.reshape(B, L, D), blk["w_o"], blk["b_o"])
+
+
+def _block_ffn(h, blk, eps):
+    """h + (silu(g) * u) W_down^T + b_down with [g | u] from RMSNorm(h)."""
+    a = rms_norm(h, blk["norm2"], eps)
+    g, u = _split(linear(a, blk["w_gu"], blk["b_gu"]), 2)
+    return h + linear(silu(g) * u, blk["w_down"], blk["b_down"])
+
+
+def denoise(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
+    """Euler denoising of the target latents ``x0[B, T, C]`` over
+    ``len(sigmas) - 1`` steps.
+
+    ``prefix_h[B, P, D]`` are the Prefix tokens' hidden states (fixed inputs);
+    ``params`` holds ``w_in[D, C]``, ``b_in[S, D]`` (one embedding bias per step:
+    the step's conditioning of the target tokens), ``blocks`` (list of dicts
+    norm1, w_qkv, b_qkv, w_o, b_o, norm2, w_gu, b_gu, w_down, b_down),
+    ``norm_out``, ``w_v[C, D]``, ``b_v``.  ``segments`` fix positions and the
+    block-causal mask (target last).  Returns x after the last step.
+    """
+    pos, kv_end = positions(segments)
+    pos = np.asarray(pos)
+    P = prefix_h.shape[1]
+    x = np.asarray(x0, dtype=np.float64)
+    prefix_h = np.asarray(prefix_h, dtype=np.float64)
+    caches = [None] * len(params["blocks"])
+    for step in range(len(sigmas) - 1):
+        h_t = linear(x, params["w_in"], params["b_in"][step])
+        if step == 0 or not cached:
+            h = np.concatenate([prefix_h, h_t], axis=1)
+            for i, blk in enumerate(params["blocks"]):
+                def attend(q, k, v, i=i):
+                    if cached:
+                        caches[i] = prefix_cache(k, v, pos, P)
+                    return attn_full(q, k, v, pos, kv_end)
+                h = _block_ffn(_block_attention(h, blk, eps, attend), blk, eps)
+            h_t = h[:, P:]
+        else:
+            h = h_t
+            for i, blk in enumerate(params["blocks"]):
+                attend = lambda q, k, v, i=i: attn_cached(q, k, v, pos[P:], caches[i][0], caches[i][1])
+                h = _block_ffn(_block_attention(h, blk, eps, attend), blk, eps)
+            h_t = h
+        vel = linear(rms_norm(h_t, params["norm_out"], eps), params["w_v"], params["b_v"])
+        x = x + (sigmas[step + 1] - sigmas[step]) * vel
+    return x
 
 
 # ----------------------------------------------------------------------------

@@ -328,12 +328,60 @@ def check_linear_special_cases(O):
     assert np.array_equal(O.linear(np.zeros((4, 8)), rng.standard_normal((3, 8)), b), np.tile(b, (4, 1)))
 
 
+# ----------------------------------------------------------- denoising loop --
+
+def _f64_params(params):
+    conv = lambda v: W.as_f64(v) if isinstance(v, torch.Tensor) else v
+    out = {k: conv(v) for k, v in params.items() if k != "blocks"}
+    out["blocks"] = [{k: conv(v) for k, v in b.items()} for b in params["blocks"]]
+    return out
+
+
+def _tiny_denoise(steps=3):
+    segs = [W.text(5), W.image(3, 3, 1), W.image(4, 4, 0)]
+    params, draw = W.denoise_model(heads=1, channels=16, blocks=2, steps=steps, seed=21, dtype="f32")
+    x0, ph = draw(1, 14, 16, 22)
+    return segs, _f64_params(params), W.as_f64(x0), W.as_f64(ph), W.denoise_sigmas(steps)
+
+
+def check_silu_vs_torch(O):
+    x = np.linspace(-30, 30, 1001)
+    ref = torch.nn.functional.silu(torch.tensor(x)).numpy()
+    assert np.max(np.abs(O.silu(x) - ref)) < 1e-13
+
+
+def check_denoise_cache_reuse(O):
+    """Overview (lab note, card 6A): reusing the Prefix K/V over the Euler steps
+    reproduces full recomputation to float64 rounding (the lab reports 1e-16)."""
+    segs, params, x0, ph, sig = _tiny_denoise()
+    xc = O.denoise(x0, ph, params, segs, sig, cached=True)
+    xf = O.denoise(x0, ph, params, segs, sig, cached=False)
+    assert np.max(np.abs(xc - xf)) < 1e-12
+    assert np.max(np.abs(xc - x0)) > 0.1  # the steps did move the latents
+
+
+def check_denoise_euler_closed_form(O):
+    """Blocks with zero weights pass h through; a constant velocity c then
+    gives x_S = x_0 + (sigma_S - sigma_0) c = x_0 - c (card 6B)."""
+    segs, params, x0, ph, sig = _tiny_denoise()
+    for blk in params["blocks"]:
+        for k in blk:
+            if not k.startswith("norm"):
+                blk[k] = np.zeros_like(blk[k])
+    params["w_v"] = np.zeros_like(params["w_v"])
+    c = np.linspace(-1, 1, params["b_v"].shape[0])
+    params["b_v"] = c
+    x = O.denoise(x0, ph, params, segs, sig, cached=True)
+    assert np.max(np.abs(x - (x0 - c))) < 1e-14
+
+
 CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_frames,
           check_prompt_length_invariance, check_block_causal_rule, check_prefix_never_sees_target,
           check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
           check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
           check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms,
-          check_linear_brute_force, check_linear_special_cases, check_original_text_offset]
+          check_linear_brute_force, check_linear_special_cases, check_original_text_offset,
+          check_silu_vs_torch, check_denoise_cache_reuse, check_denoise_euler_closed_form]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
@@ -467,6 +515,23 @@ def _original_from_zero(segments):
     return OM.positions(segments)[0], kv
 
 
+def _silu_as_sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-np.asarray(x, dtype=np.float64)))
+
+
+def _denoise_step_sign(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
+    return OM.denoise(x0, prefix_h, params, segments, [-s for s in sigmas], cached, eps)
+
+
+def _denoise_stale_target(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
+    """A cached loop that drifts from the full recomputation: its later steps
+    only go half way."""
+    if not cached:
+        return OM.denoise(x0, prefix_h, params, segments, sigmas, False, eps)
+    x = OM.denoise(x0, prefix_h, params, segments, sigmas[:2], True, eps)
+    return x + (OM.denoise(x, prefix_h, params, segments, sigmas[1:], False, eps) - x) * 0.5
+
+
 MUTANTS = {
     "rope_sign": dict(rope=_rope_sign_flipped),
     "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
@@ -482,6 +547,9 @@ MUTANTS = {
     "linear_bias_dropped": dict(linear=_linear_no_bias),
     "original_offset_unhalved": dict(positions_original=_original_offset_unhalved),
     "original_text_from_zero": dict(positions_original=_original_from_zero),
+    "silu_as_sigmoid": dict(silu=_silu_as_sigmoid),
+    "euler_step_sign": dict(denoise=_denoise_step_sign),
+    "cache_not_reused_faithfully": dict(denoise=_denoise_stale_target),
 }
 
 
