@@ -274,6 +274,67 @@ def time_projections(qi, args, M, D, flush, dev):
     return out
 
 
+def time_denoise(qi, args, cfg, dev):
+    """The denoising loop around the attention on this workload's layout:
+    ``--denoise-blocks`` blocks (attention + SwiGLU), 8 Euler steps, random
+    weights drawn on the device (N(0, 1/fan_in); biases 0.02 N(0, 1)), 64
+    latent channels.  One graph replay = one whole loop (step 1 on every
+    token, steps 2..8 on the target tokens against the per-block caches).
+    Also runs the full recomputation once from the same latents and reports
+    the largest difference (the cache-reuse check)."""
+    steps, C, nb, H = 8, 64, args.denoise_blocks, cfg["H"]
+    sig = W.denoise_sigmas(steps)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(13)
+    D, F = H * 128, 3 * H * 128
+    rnd = lambda *shape, scale=1.0, shift=0.0: (torch.randn(*shape, generator=gen, device=dev) * scale
+                                                 + shift).to(torch.bfloat16)
+    blk = lambda: dict(norm1=rnd(D, scale=0.1, shift=1.0), w_qkv=rnd(3 * D, D, scale=D ** -0.5),
+                       b_qkv=rnd(3 * D, scale=0.02), w_o=rnd(D, D, scale=D ** -0.5), b_o=rnd(D, scale=0.02),
+                       norm2=rnd(D, scale=0.1, shift=1.0), w_gu=rnd(2 * F, D, scale=D ** -0.5),
+                       b_gu=rnd(2 * F, scale=0.02), w_down=rnd(D, F, scale=F ** -0.5), b_down=rnd(D, scale=0.02))
+    params = dict(w_in=rnd(D, C, scale=C ** -0.5), b_in=rnd(steps, D, scale=0.5), blocks=[blk() for _ in range(nb)],
+                  norm_out=rnd(D, scale=0.1, shift=1.0), w_v=rnd(C, D, scale=D ** -0.5), b_v=rnd(C, scale=0.02))
+    segs = cfg["segments"]
+    L = sum(W.seg_tokens(s) for s in segs)
+    T = W.seg_tokens(segs[-1])
+    x0, ph = rnd(1, T, C), rnd(1, L - T, D)
+    model = qi.denoise.DenoiseModel(segs, H, C, nb, steps, sig, device=dev, cached=True)
+    model.load(params, x0, ph)
+    model.run()
+    model.check()
+    x_cached = model.x.clone()
+    model.x.copy_(x0)
+    model.capture()
+    reps = max(2, min(args.steps, 5))
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps + 1)]
+    for i, (a, b) in enumerate(ev):  # the first replay is a warm-up
+        a.record(stream)
+        model.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    model.check()
+    ms = pct([a.elapsed_time(b) for a, b in ev[1:]], 50)
+    flops = model.flops()
+    del model
+    torch.cuda.empty_cache()
+    full = qi.denoise.DenoiseModel(segs, H, C, nb, steps, sig, device=dev, cached=False)
+    full.load(params, x0, ph)
+    full.run()
+    full.check()
+    diff = (full.x.float() - x_cached.float()).abs()
+    out = {"blocks": nb, "steps": steps, "heads": H, "channels": C, "tokens": L, "target_tokens": T,
+           "graph_ms_median": ms, "tflop_per_loop": flops / 1e12, "tflops": flops / (ms * 1e-3) / 1e12,
+           "cached_vs_full_max_abs": float(diff.max()), "cached_vs_full_mean_abs": float(diff.mean()),
+           "latent_rms": float(x_cached.float().pow(2).mean().sqrt()),
+           "what": "reduced loop: embedding, blocks of RMSNorm/attention/SwiGLU with residuals, velocity, "
+                   "Euler; random weights on the device"}
+    del full
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops):
     """The workload's denoising loop for one layer: step 1 full (cache store)
     and steps 2..N cached on fresh target inputs, timed eagerly (one library
@@ -442,6 +503,9 @@ def run_ours(args, world, rank, local):
     if cfg.get("cached_steps", 0) > 1 and not args.qk_norm:
         loop = time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops)
 
+    # ---- the whole denoising loop around the attention (optional: heavy)
+    dn = time_denoise(qi, args, cfg, dev) if args.denoise and not cfg.get("original") else None
+
     # ---- end to end through the C ABI with host buffers (copies timed)
     h2d = sum(x.numel() * x.element_size() for x in host)
     outs_d = [o_full] if orig else [o_full, o_c]
@@ -523,6 +587,8 @@ def run_ours(args, world, rank, local):
         "clocks": clk,
     }
     line["projections"] = proj
+    if dn is not None:
+        line["denoise"] = dn
     if loop is not None:
         line["loop"] = loop
     print(json.dumps(line), flush=True)
@@ -537,6 +603,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--denoise", action="store_true",
+                    help="also time the whole denoising loop (blocks of attention + SwiGLU, 8 Euler steps)")
+    ap.add_argument("--denoise-blocks", type=int, default=32)
     ap.add_argument("--qk-norm", action="store_true",
                     help="time the variant with the QK-RMSNorm fused in front of RoPE")
     args = ap.parse_args(argv)

@@ -6,12 +6,14 @@ behind a C ABI (``include/qi21.h``).  This package is the thin Python
 binding: it marshals torch tensors into that ABI and nothing else.
 """
 
-from ._binding import (QI21Error, Segment, alloc_cache, attn_cached, attn_full, cached_workspace_size,
-                       full_workspace_size, launch_count, linear, load_library, new_workspace, rope_positions,
-                       selftest_exp2, selftest_wait_timeout, time_next_attention, workspace_status, HEAD_DIM,
-                       LIB_PATH)
+from ._binding import (HEAD_DIM, LIB_PATH, QI21Error, Segment, alloc_cache, attn_cached, attn_full,
+                       cached_workspace_size, full_workspace_size, launch_count, linear, linear_residual,
+                       load_library, new_workspace, rmsnorm, rope_positions, selftest_exp2,
+                       selftest_wait_timeout, swiglu, time_next_attention, workspace_status)
+from . import denoise
 from .steploop import DenoiseLoop
 
-__all__ = ["DenoiseLoop", "QI21Error", "Segment", "alloc_cache", "attn_cached", "attn_full", "cached_workspace_size",
-           "full_workspace_size", "launch_count", "linear", "load_library", "new_workspace", "rope_positions",
-           "selftest_exp2", "selftest_wait_timeout", "time_next_attention", "workspace_status", "HEAD_DIM", "LIB_PATH"]
+__all__ = ["DenoiseLoop", "HEAD_DIM", "LIB_PATH", "QI21Error", "Segment", "alloc_cache", "attn_cached",
+           "attn_full", "cached_workspace_size", "full_workspace_size", "launch_count", "linear",
+           "linear_residual", "load_library", "new_workspace", "rmsnorm", "rope_positions", "selftest_exp2",
+           "selftest_wait_timeout", "swiglu", "time_next_attention", "workspace_status"]

@@ -28,7 +28,8 @@ EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_f
             "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
             "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
-            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear", "qi21_rope_positions_original")
+            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear", "qi21_rope_positions_original",
+            "qi21_linear_residual", "qi21_rmsnorm", "qi21_swiglu")
 
 
 class QI21Error(RuntimeError):
@@ -75,6 +76,12 @@ def load_library(path=LIB_PATH):
                                           _vp, _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
     L.qi21_linear.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, ctypes.POINTER(_vp), _i32, _vp, _sz, _vp]
     L.qi21_linear.restype = _i32
+    L.qi21_linear_residual.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _sz, _vp]
+    L.qi21_linear_residual.restype = _i32
+    L.qi21_rmsnorm.argtypes = [_i64, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]
+    L.qi21_rmsnorm.restype = _i32
+    L.qi21_swiglu.argtypes = [_i64, _vp, _vp, _vp, _vp]
+    L.qi21_swiglu.restype = _i32
     L.qi21_workspace_status.argtypes = [_vp, _vp]
     L.qi21_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
     L.qi21_status_string.argtypes = [_i32]
@@ -314,6 +321,64 @@ def linear(x, w, bias=None, n_out=1, out=None, workspace=None):
     with torch.cuda.device(dev):
         _check(L_.qi21_linear(M, N, K, _ptr(x), _ptr(w), _ptr(bias), ptrs, n_out, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(dev)))
+    return out
+
+
+def linear_residual(x, w, bias, residual, alpha=1.0, out=None, workspace=None):
+    """out = residual + alpha * (x W^T + b) on the tensor cores (bf16).
+
+    x: [..., K], w: [N, K], bias: [N] or None, residual: [..., N]; ``out``
+    defaults to a new tensor and may be ``residual`` itself."""
+    L_ = _cuda_lib()
+    dev = x.device
+    K, N = x.shape[-1], w.shape[0]
+    lead = tuple(x.shape[:-1])
+    M = 1
+    for d in lead:
+        M *= int(d)
+    _need(x, "x", lead + (K,), torch.bfloat16, dev)
+    _need(w, "w", (N, K), torch.bfloat16, dev)
+    if bias is not None:
+        _need(bias, "bias", (N,), torch.bfloat16, dev)
+    _need(residual, "residual", lead + (N,), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty_like(residual)
+    _need(out, "out", lead + (N,), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(WORKSPACE_HEADER_BYTES, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_linear_residual(M, N, K, _ptr(x), _ptr(w), _ptr(bias), _ptr(residual),
+                                       ctypes.c_float(float(alpha)), _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(dev)))
+    return out
+
+
+def rmsnorm(x, w, eps, out=None):
+    """Row RMSNorm over the last axis (bf16): x / sqrt(mean(x^2) + eps) * w."""
+    L_ = _cuda_lib()
+    dev, D = x.device, x.shape[-1]
+    _need(x, "x", tuple(x.shape), torch.bfloat16, dev)
+    _need(w, "w", (D,), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", tuple(x.shape), torch.bfloat16, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_rmsnorm(x.numel() // D, D, _ptr(x), _ptr(w), ctypes.c_float(float(eps)), _ptr(out),
+                               _stream(dev)))
+    return out
+
+
+def swiglu(g, u, out=None):
+    """silu(g) * u elementwise (bf16)."""
+    L_ = _cuda_lib()
+    dev = g.device
+    _need(g, "g", tuple(g.shape), torch.bfloat16, dev)
+    _need(u, "u", tuple(g.shape), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty_like(g)
+    _need(out, "out", tuple(g.shape), torch.bfloat16, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_swiglu(g.numel(), _ptr(g), _ptr(u), _ptr(out), _stream(dev)))
     return out
 
 

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqi21.so")
-SOURCES = ["api.cu", "prep_kernels.cu", "attn_simt.cu", "attn_tc.cu", "gemm_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "prep_kernels.cu", "attn_simt.cu", "attn_tc.cu", "gemm_tc.cu", "rowwise.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -375,9 +375,9 @@ qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, 
                           workspace, workspace_bytes, stream);
 }
 
-qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
-                        void* const* out, int32_t n_out, void* workspace, size_t workspace_bytes,
-                        void* stream) {
+static qi21_status linear_impl(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
+                               void* const* out, int32_t n_out, const void* residual, float alpha,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   if (M < 0 || N < 0 || K < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
     return fail(QI21_ERR_INVALID_ARG, "M, N, K must be in [0, 2^31)");
   if (n_out < 1 || n_out > 4) return fail(QI21_ERR_INVALID_ARG, "n_out must be in [1, 4] (got %d)", n_out);
@@ -406,9 +406,53 @@ qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const vo
   a.bias = bias;
   for (int i = 0; i < n_out; ++i) a.out[i] = out[i];
   a.n_out = n_out;
+  a.residual = residual;
+  a.alpha = alpha;
   a.status = static_cast<uint32_t*>(workspace);
   cudaError_t e = launch_gemm_tc(a, static_cast<cudaStream_t>(stream), sm_count());
   if (e != cudaSuccess) return cuda_fail(e, "linear launch");
+  return QI21_OK;
+}
+
+qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
+                        void* const* out, int32_t n_out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return linear_impl(M, N, K, x, w, bias, out, n_out, nullptr, 1.0f, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_linear_residual(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                                 const void* bias, const void* residual, float alpha, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (M > 0 && N > 0) QI21_TRY(check_ptr(residual, "residual"));
+  if (!(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f)
+    return fail(QI21_ERR_INVALID_ARG, "alpha must be finite");
+  void* outs[1] = {out};
+  return linear_impl(M, N, K, x, w, bias, outs, 1, residual, alpha, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_rmsnorm(int64_t M, int32_t D, const void* x, const void* w, float eps, void* y,
+                         void* stream) {
+  if (M < 0 || D < 8 || D % 8 != 0 || M > INT32_MAX)
+    return fail(QI21_ERR_INVALID_ARG, "need M >= 0 and D a multiple of 8 (M=%lld, D=%d)", (long long)M, D);
+  if (!(eps >= 0.f) || !(eps < 3.0e38f)) return fail(QI21_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (M == 0) return QI21_OK;
+  QI21_TRY(check_ptr(x, "x"));
+  QI21_TRY(check_ptr(w, "w"));
+  QI21_TRY(check_ptr(y, "y"));
+  cudaError_t e = launch_rmsnorm(M, D, x, w, eps, y, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  return QI21_OK;
+}
+
+qi21_status qi21_swiglu(int64_t n, const void* g, const void* u, void* m, void* stream) {
+  if (n < 0 || n % 8 != 0 || n / 8 > INT32_MAX)
+    return fail(QI21_ERR_INVALID_ARG, "n must be a non-negative multiple of 8 (got %lld)", (long long)n);
+  if (n == 0) return QI21_OK;
+  QI21_TRY(check_ptr(g, "g"));
+  QI21_TRY(check_ptr(u, "u"));
+  QI21_TRY(check_ptr(m, "m"));
+  cudaError_t e = launch_swiglu(n, g, u, m, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "swiglu launch");
   return QI21_OK;
 }
 

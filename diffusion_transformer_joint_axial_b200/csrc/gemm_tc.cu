@@ -16,7 +16,8 @@
 // Roles (256 threads):
 //   warp 0     TMA producer: a 4-stage ring of (X 128x64, W 256x64) K-steps
 //   warp 1     TMEM owner and tcgen05.mma issuer (M=128, N=256, K=16)
-//   warps 4-7  epilogue: TMEM -> fp32 (+ bias) -> bf16 -> global, row per thread
+//   warps 4-7  epilogue: TMEM -> fp32 (+ bias, or residual + alpha * (. + bias))
+//              -> bf16 -> global, row per thread
 // TMEM holds two 256-column fp32 accumulators, so the epilogue of one tile
 // overlaps the MMAs of the next.  Rows, columns and K past the end are
 // zero-filled by TMA and never stored.  Every wait is bounded.
@@ -54,6 +55,8 @@ struct Params {
   int32_t mt, nt, kt;           // tiles along M, N and K steps
   __nv_bfloat16* out[kMaxOut];  // [M, n_seg] each
   const __nv_bfloat16* bias;    // [N] or null
+  const __nv_bfloat16* residual;  // [M, N] added to alpha * (X W^T + b), or null (may be out[0])
+  float alpha;
   uint32_t* status;
 };
 
@@ -226,6 +229,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             const int seg = col / p.n_seg;
             __nv_bfloat16* dst = p.out[seg] + (size_t)row * p.n_seg + (col - seg * p.n_seg);
+            if (p.residual != nullptr) {
+              // the same thread reads this residual chunk and then writes the
+              // output chunk, so the residual may be the output itself
+              const uint4 rr = *reinterpret_cast<const uint4*>(p.residual + (size_t)row * p.N + col);
+              const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rr);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 rf = unpack_bf16x2(rw[e]);
+                f[2 * e] = fmaf(p.alpha, f[2 * e], rf.x);
+                f[2 * e + 1] = fmaf(p.alpha, f[2 * e + 1], rf.y);
+              }
+            }
             *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                                         pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
           }
@@ -287,6 +302,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms) 
   p.kt = (int32_t)((a.K + gemm::BK - 1) / gemm::BK);
   for (int i = 0; i < a.n_out; ++i) p.out[i] = static_cast<__nv_bfloat16*>(a.out[i]);
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
+  p.residual = static_cast<const __nv_bfloat16*>(a.residual);
+  p.alpha = a.alpha;
   p.status = a.status;
   const size_t smem = sizeof(gemm::Smem) + 1024;
   cudaError_t err =

@@ -104,9 +104,18 @@ struct GemmArgs {
   const void* bias;
   void* out[4];
   int32_t n_out;
+  const void* residual;  // [M, N]: out = residual + alpha * (X W^T + b) (n_out = 1), or null
+  float alpha;
   uint32_t* status;  // workspace header status word
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);
+
+// ---------------------------------------------------------- row-wise ops
+// y = x / sqrt(mean(x^2) + eps) * w over rows of D (bf16), one warp per row.
+cudaError_t launch_rmsnorm(int64_t M, int32_t D, const void* x, const void* w, float eps, void* y,
+                           cudaStream_t stream);
+// m = silu(g) * u elementwise (bf16, n a multiple of 8).
+cudaError_t launch_swiglu(int64_t n, const void* g, const void* u, void* m, cudaStream_t stream);
 
 // --------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);

@@ -224,6 +224,33 @@ qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const vo
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The rest of a block of the denoising loop around the attention (overview
+ * cards 4A and 5A: each of the stacked blocks runs attention, then a SwiGLU
+ * feed-forward layer 3x wider than the model, each behind an RMSNorm and
+ * added back to the residual stream; card 6B: the Euler step).
+ *
+ * qi21_linear_residual -- out = residual + alpha * (X W^T + b): qi21_linear
+ *   with one output and a residual added in its epilogue (a residual
+ *   connection with alpha = 1; the Euler step x + (sigma' - sigma) v with the
+ *   velocity head as the projection).  residual: device bf16 [M, N], 16-byte
+ *   aligned; it may be out itself (each element is read before it is
+ *   written, by the same thread).  alpha finite.
+ */
+qi21_status qi21_linear_residual(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                                 const void* bias, const void* residual, float alpha, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* qi21_rmsnorm -- y = x / sqrt(mean(x^2) + eps) * w over each of the M rows
+ * of D values (bf16 x, w [D], y; D a multiple of 8; 16-byte aligned; eps
+ * finite, >= 0).  y may not overlap x. */
+qi21_status qi21_rmsnorm(int64_t M, int32_t D, const void* x, const void* w, float eps, void* y,
+                         void* stream);
+
+/* qi21_swiglu -- m = silu(g) * u elementwise, silu(g) = g / (1 + exp(-g)),
+ * over n bf16 values (n a multiple of 8; 16-byte aligned; m may be g or u). */
+qi21_status qi21_swiglu(int64_t n, const void* g, const void* u, void* m, void* stream);
+
+/*
  * qi21_attn_cached_noalloc -- the cached step of qi21_attn_cached for callers
  * that may not allocate device memory (plugin hosts that only hand over a
  * stream and tensors, servers that reserve all memory at start-up, loops where

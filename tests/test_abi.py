@@ -168,6 +168,24 @@ def test_linear_rejects(lib):
     assert lin(M=0, x=None, w=None, ws=None) == qb.QI21_OK  # nothing to do
 
 
+def test_block_ops_reject(lib):
+    p = ctypes.c_void_p
+    bad = qb.QI21_ERR_INVALID_ARG
+    lr = lambda residual=16, alpha=1.0, N=64: lib.qi21_linear_residual(
+        32, N, 64, p(16), p(16), None, p(residual) if residual else None, ctypes.c_float(alpha), p(16),
+        p(256), 256, None)
+    assert lr(residual=None) == bad and lr(residual=24) == bad   # missing / misaligned residual
+    assert lr(alpha=float("nan")) == bad and lr(alpha=float("inf")) == bad
+    assert lr(N=60) == bad                                        # N not a multiple of 8
+    rn = lambda M=4, D=64, eps=1e-6, x=16: lib.qi21_rmsnorm(M, D, p(x) if x else None, p(16), ctypes.c_float(eps),
+                                                           p(16), None)
+    assert rn(D=60) == bad and rn(D=0) == bad and rn(eps=-1.0) == bad and rn(x=None) == bad
+    assert rn(M=0, x=None) == qb.QI21_OK
+    sw = lambda n=64, g=16: lib.qi21_swiglu(n, p(g) if g else None, p(16), p(16), None)
+    assert sw(n=60) == bad and sw(n=-8) == bad and sw(g=None) == bad and sw(g=8) == bad
+    assert sw(n=0, g=None) == qb.QI21_OK
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.qi21_selftest_wait_timeout(ctypes.c_void_p(256), 0, None) == qb.QI21_ERR_INVALID_ARG
 
