@@ -46,6 +46,7 @@ def _check(got, x, w, b, rows=None, what=""):
     (256, 512, 128, 1, True),     # exact tiles
     (130, 264, 72, 1, False),     # one row and one column group past a tile
     (300, 1024, 512, 4, True),    # four segments
+    (1000, 20480, 136, 2, True),  # many column tiles, ragged in M and K
 ])
 def test_linear_shapes(cuda_device, M, N, K, n_out, bias):
     x, w, b = _draw(M, N, K, seed=M + N + K, bias=bias)
