@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // The whole warp runs the loop (every value is warp-uniform, so the
       // TMA operands stay in uniform registers); one elected lane issues.
       const bool leader = elect_one_sync();
-      uint32_t kc = 0, vc = 0, ql[2] = {0, 0};
+      uint32_t kc = 0, vc = 0, ql[2] = {0, 0}, qi[2] = {0, 0};
       bool ok = true;
       while (ok) {
         if (do_qk) publish_unit(S, p, sc, leader, abort_flag, ok);
@@ -411,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_empty[s]), (ql[s] & 1u) ^ 1u,
                                                 abort_flag, p.status, 0x100 | s));
           ++ql[s];
+          if (ok) ++qi[s];  // Q loads issued into buffer s
           if (ok && leader) {
             const uint32_t bar = smem_u32(&S.q_full[s]);
             mbar_arrive_expect_tx(bar, kTileBytes);
@@ -452,6 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // Every load this warp issued lands before the CTA may exit: wait
       // (bounded) for the last load issued into each stage.
       if (!ok) {
+        for (int s = 0; s < 2 && do_qk; ++s)
+          if (qi[s] > 0) mbar_wait(smem_u32(&S.q_full[s]), (qi[s] - 1) & 1u, nullptr, nullptr, 0);
         for (uint32_t st = 0; st < kStages; ++st) {
           if (kc > st) {
             const uint32_t last = ((kc - 1 - st) / kStages) * kStages + st;
