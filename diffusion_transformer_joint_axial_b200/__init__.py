@@ -7,13 +7,14 @@ binding: it marshals torch tensors into that ABI and nothing else.
 """
 
 from ._binding import (HEAD_DIM, LIB_PATH, QI21Error, Segment, alloc_cache, attn_cached, attn_full,
-                       cached_workspace_size, full_workspace_size, launch_count, linear, linear_residual,
+                       cached_workspace_size, full_workspace_size, interleave_gate_up, launch_count, linear,
+                       linear_residual, linear_swiglu,
                        load_library, new_workspace, rmsnorm, rope_positions, selftest_exp2,
                        selftest_wait_timeout, swiglu, time_next_attention, workspace_status)
 from . import denoise
 from .steploop import DenoiseLoop
 
 __all__ = ["DenoiseLoop", "HEAD_DIM", "LIB_PATH", "QI21Error", "Segment", "alloc_cache", "attn_cached",
-           "attn_full", "cached_workspace_size", "full_workspace_size", "launch_count", "linear",
-           "linear_residual", "load_library", "new_workspace", "rmsnorm", "rope_positions", "selftest_exp2",
+           "attn_full", "cached_workspace_size", "full_workspace_size", "interleave_gate_up", "launch_count",
+           "linear", "linear_residual", "linear_swiglu", "load_library", "new_workspace", "rmsnorm", "rope_positions", "selftest_exp2",
            "selftest_wait_timeout", "swiglu", "time_next_attention", "workspace_status"]

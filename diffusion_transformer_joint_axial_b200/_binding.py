@@ -29,7 +29,7 @@ EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_f
             "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
             "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
             "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear", "qi21_rope_positions_original",
-            "qi21_linear_residual", "qi21_rmsnorm", "qi21_swiglu")
+            "qi21_linear_residual", "qi21_rmsnorm", "qi21_swiglu", "qi21_linear_swiglu")
 
 
 class QI21Error(RuntimeError):
@@ -78,6 +78,8 @@ def load_library(path=LIB_PATH):
     L.qi21_linear.restype = _i32
     L.qi21_linear_residual.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _sz, _vp]
     L.qi21_linear_residual.restype = _i32
+    L.qi21_linear_swiglu.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    L.qi21_linear_swiglu.restype = _i32
     L.qi21_rmsnorm.argtypes = [_i64, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]
     L.qi21_rmsnorm.restype = _i32
     L.qi21_swiglu.argtypes = [_i64, _vp, _vp, _vp, _vp]
@@ -350,6 +352,41 @@ def linear_residual(x, w, bias, residual, alpha=1.0, out=None, workspace=None):
         _check(L_.qi21_linear_residual(M, N, K, _ptr(x), _ptr(w), _ptr(bias), _ptr(residual),
                                        ctypes.c_float(float(alpha)), _ptr(out), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(dev)))
+    return out
+
+
+def interleave_gate_up(t):
+    """[gate; up] stacked along dim 0 (2F rows, or a 2F bias) -> the
+    alternating 128-row blocks qi21_linear_swiglu reads (F a multiple of 128)."""
+    F = t.shape[0] // 2
+    rest = tuple(t.shape[1:])
+    return t.reshape((2, F // 128, 128) + rest).transpose(0, 1).reshape((2 * F,) + rest).contiguous()
+
+
+def linear_swiglu(x, w_il, bias_il=None, out=None, workspace=None):
+    """silu(x W_gate^T + b_gate) * (x W_up^T + b_up) in one tensor-core launch.
+
+    ``w_il`` [2F, K] and ``bias_il`` [2F] in the layout of
+    :func:`interleave_gate_up`; returns [..., F]."""
+    L_ = _cuda_lib()
+    dev = x.device
+    K, N = x.shape[-1], w_il.shape[0]
+    lead = tuple(x.shape[:-1])
+    M = 1
+    for d in lead:
+        M *= int(d)
+    _need(x, "x", lead + (K,), torch.bfloat16, dev)
+    _need(w_il, "w", (N, K), torch.bfloat16, dev)
+    if bias_il is not None:
+        _need(bias_il, "bias", (N,), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty(lead + (N // 2,), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", lead + (N // 2,), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(WORKSPACE_HEADER_BYTES, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_linear_swiglu(M, N, K, _ptr(x), _ptr(w_il), _ptr(bias_il), _ptr(out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(dev)))
     return out
 
 

@@ -377,7 +377,7 @@ qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, 
 
 static qi21_status linear_impl(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
                                void* const* out, int32_t n_out, const void* residual, float alpha,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               bool swiglu, void* workspace, size_t workspace_bytes, void* stream) {
   if (M < 0 || N < 0 || K < 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
     return fail(QI21_ERR_INVALID_ARG, "M, N, K must be in [0, 2^31)");
   if (n_out < 1 || n_out > 4) return fail(QI21_ERR_INVALID_ARG, "n_out must be in [1, 4] (got %d)", n_out);
@@ -408,6 +408,7 @@ static qi21_status linear_impl(int64_t M, int64_t N, int64_t K, const void* x, c
   a.n_out = n_out;
   a.residual = residual;
   a.alpha = alpha;
+  a.swiglu = swiglu ? 1 : 0;
   a.status = static_cast<uint32_t*>(workspace);
   cudaError_t e = launch_gemm_tc(a, static_cast<cudaStream_t>(stream), sm_count());
   if (e != cudaSuccess) return cuda_fail(e, "linear launch");
@@ -417,7 +418,8 @@ static qi21_status linear_impl(int64_t M, int64_t N, int64_t K, const void* x, c
 qi21_status qi21_linear(int64_t M, int64_t N, int64_t K, const void* x, const void* w, const void* bias,
                         void* const* out, int32_t n_out, void* workspace, size_t workspace_bytes,
                         void* stream) {
-  return linear_impl(M, N, K, x, w, bias, out, n_out, nullptr, 1.0f, workspace, workspace_bytes, stream);
+  return linear_impl(M, N, K, x, w, bias, out, n_out, nullptr, 1.0f, false, workspace, workspace_bytes,
+                     stream);
 }
 
 qi21_status qi21_linear_residual(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
@@ -427,7 +429,17 @@ qi21_status qi21_linear_residual(int64_t M, int64_t N, int64_t K, const void* x,
   if (!(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f)
     return fail(QI21_ERR_INVALID_ARG, "alpha must be finite");
   void* outs[1] = {out};
-  return linear_impl(M, N, K, x, w, bias, outs, 1, residual, alpha, workspace, workspace_bytes, stream);
+  return linear_impl(M, N, K, x, w, bias, outs, 1, residual, alpha, false, workspace, workspace_bytes, stream);
+}
+
+qi21_status qi21_linear_swiglu(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                               const void* bias, void* out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (N % 256 != 0)
+    return fail(QI21_ERR_INVALID_ARG, "N must be a multiple of 256 (gate/up blocks of 128; got %lld)",
+                (long long)N);
+  void* outs[1] = {out};
+  return linear_impl(M, N, K, x, w, bias, outs, 1, nullptr, 1.0f, true, workspace, workspace_bytes, stream);
 }
 
 qi21_status qi21_rmsnorm(int64_t M, int32_t D, const void* x, const void* w, float eps, void* y,

@@ -16,8 +16,9 @@
 // Roles (256 threads):
 //   warp 0     TMA producer: a 4-stage ring of (X 128x64, W 256x64) K-steps
 //   warp 1     TMEM owner and tcgen05.mma issuer (M=128, N=256, K=16)
-//   warps 4-7  epilogue: TMEM -> fp32 (+ bias, or residual + alpha * (. + bias))
-//              -> bf16 -> global, row per thread
+//   warps 4-7  epilogue: TMEM -> fp32 (+ bias, or residual + alpha * (. + bias),
+//              or silu(gate) * up of a tile's two column halves) -> bf16 -> global,
+//              row per thread
 // TMEM holds two 256-column fp32 accumulators, so the epilogue of one tile
 // overlaps the MMAs of the next.  Rows, columns and K past the end are
 // zero-filled by TMA and never stored.  Every wait is bounded.
@@ -57,6 +58,7 @@ struct Params {
   const __nv_bfloat16* bias;    // [N] or null
   const __nv_bfloat16* residual;  // [M, N] added to alpha * (X W^T + b), or null (may be out[0])
   float alpha;
+  int32_t swiglu;  // 1: W holds gate/up rows in alternating 128-row blocks; out[0] = silu(gate) * up
   uint32_t* status;
 };
 
@@ -204,6 +206,51 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       tc_fence_after();
       const int row = (t % p.mt) * BM + r;
       const int n0 = (t / p.mt) * BN;
+      if (p.swiglu) {
+        // columns [0, 128) of the tile are the gates of output features
+        // n0/2 + [0, 128), columns [128, 256) their up projections
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(tmem + lane_base + buf * BN + c, gv);
+          tmem_ld32(tmem + lane_base + buf * BN + BN / 2 + c, uv);
+          tmem_wait_ld();
+          if (row < p.M) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float gate[8], up[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                gate[e] = __uint_as_float(gv[8 * g + e]);
+                up[e] = __uint_as_float(uv[8 * g + e]);
+              }
+              if (p.bias != nullptr) {
+                const uint4 bg = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + c + 8 * g));
+                const uint4 bu = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + BN / 2 + c + 8 * g));
+                const uint32_t* bgw = reinterpret_cast<const uint32_t*>(&bg);
+                const uint32_t* buw = reinterpret_cast<const uint32_t*>(&bu);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 a = unpack_bf16x2(bgw[e]), b = unpack_bf16x2(buw[e]);
+                  gate[2 * e] += a.x;
+                  gate[2 * e + 1] += a.y;
+                  up[2 * e] += b.x;
+                  up[2 * e + 1] += b.y;
+                }
+              }
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = gate[e] / (1.f + expf(-gate[e])) * up[e];
+              __nv_bfloat16* dst = p.out[0] + (size_t)row * p.n_seg + n0 / 2 + c + 8 * g;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&S.acc_empty[buf]));
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32];
@@ -296,7 +343,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms) 
   p.M = (int32_t)a.M;
   p.N = (int32_t)a.N;
   p.K = (int32_t)a.K;
-  p.n_seg = (int32_t)(a.N / a.n_out);
+  p.n_seg = (int32_t)(a.swiglu ? a.N / 2 : a.N / a.n_out);
+  p.swiglu = a.swiglu;
   p.mt = (int32_t)((a.M + gemm::BM - 1) / gemm::BM);
   p.nt = (int32_t)((a.N + gemm::BN - 1) / gemm::BN);
   p.kt = (int32_t)((a.K + gemm::BK - 1) / gemm::BK);

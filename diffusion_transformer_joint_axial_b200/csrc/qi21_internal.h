@@ -106,6 +106,8 @@ struct GemmArgs {
   int32_t n_out;
   const void* residual;  // [M, N]: out = residual + alpha * (X W^T + b) (n_out = 1), or null
   float alpha;
+  int32_t swiglu;        // 1: gate/up rows of W alternate in 128-row blocks; out[0] [M, N/2]
+                         //    = silu(gate) * up (n_out = 1, N a multiple of 256)
   uint32_t* status;  // workspace header status word
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);

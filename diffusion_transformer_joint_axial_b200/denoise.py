@@ -16,8 +16,9 @@ step -- holds as in the full model.  One batch element (B = 1).  Parameters
 are those of ``workloads.denoise_model`` (the oracle's ``denoise`` layout).
 
 This module is plumbing: it allocates buffers once and enqueues library
-calls (projections, RMSNorm, SwiGLU, RoPE/cache pre-pass, attention) in
-stream order; every arithmetic step runs in libqi21's kernels.
+calls (projections, RMSNorm, the projection with the SwiGLU gate in its
+epilogue, RoPE/cache pre-pass, attention) in stream order; every arithmetic
+step runs in libqi21's kernels.
 """
 
 import torch
@@ -69,7 +70,7 @@ class DenoiseModel:
         z = lambda *shape: torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
         D, F, H = self.D, self.F, self.H
         return dict(h=z(1, n, D), a=z(1, n, D), q=z(1, n, H, 128), k=z(1, n, H, 128), v=z(1, n, H, 128),
-                    o=z(1, n, H, 128), g=z(1, n, F), u=z(1, n, F), m=z(1, n, F))
+                    o=z(1, n, H, 128), m=z(1, n, F))
 
     def load(self, params, x0, prefix_h):
         """Copies parameters (``workloads.denoise_model`` layout), the initial
@@ -80,6 +81,11 @@ class DenoiseModel:
             pairs += [(mine[k], theirs[k]) for k in mine]
         for dst, src in pairs:
             dst.copy_(src, non_blocking=True)
+        # the feed-forward layer's [gate; up] weights go to the alternating
+        # 128-row blocks of the fused projection + SwiGLU launch
+        for blk in self.blocks:
+            blk["w_gu"].copy_(qb.interleave_gate_up(blk["w_gu"]))
+            blk["b_gu"].copy_(qb.interleave_gate_up(blk["b_gu"]))
 
     def _block(self, i, A, n):
         """One block on the n tokens of activation set A."""
@@ -97,8 +103,7 @@ class DenoiseModel:
             qb.attn_cached(A["q"], A["k"], A["v"], self.pos_t, kc, vc, out=A["o"], workspace=self.ws_cached)
         qb.linear_residual(flat(A["o"]), blk["w_o"], blk["b_o"], A["h"], out=A["h"], workspace=ws)
         qb.rmsnorm(A["h"], blk["norm2"], self.eps, out=A["a"])
-        qb.linear(A["a"], blk["w_gu"], blk["b_gu"], n_out=2, out=[A["g"], A["u"]], workspace=ws)
-        qb.swiglu(A["g"], A["u"], out=A["m"])
+        qb.linear_swiglu(A["a"], blk["w_gu"], blk["b_gu"], out=A["m"], workspace=ws)
         qb.linear_residual(A["m"], blk["w_down"], blk["b_down"], A["h"], out=A["h"], workspace=ws)
 
     def run(self):

@@ -240,6 +240,19 @@ qi21_status qi21_linear_residual(int64_t M, int64_t N, int64_t K, const void* x,
                                  const void* bias, const void* residual, float alpha, void* out,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * qi21_linear_swiglu -- out = silu(X W_gate^T + b_gate) * (X W_up^T + b_up)
+ *   in one launch: the feed-forward layer's gated first half (card 5A) with
+ *   the gate in the projection's epilogue.  W ([N, K]) and bias ([N]) hold
+ *   the gate and up rows in alternating blocks of 128: rows 256j..256j+127 are
+ *   the gates of output features 128j..128j+127, rows 256j+128..256j+255 their
+ *   up projections.  N a multiple of 256; out: device bf16 [M, N / 2].  Other
+ *   arguments and errors as for qi21_linear.
+ */
+qi21_status qi21_linear_swiglu(int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                               const void* bias, void* out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* qi21_rmsnorm -- y = x / sqrt(mean(x^2) + eps) * w over each of the M rows
  * of D values (bf16 x, w [D], y; D a multiple of 8; 16-byte aligned; eps
  * finite, >= 0).  y may not overlap x. */

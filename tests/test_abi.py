@@ -181,6 +181,8 @@ def test_block_ops_reject(lib):
                                                            p(16), None)
     assert rn(D=60) == bad and rn(D=0) == bad and rn(eps=-1.0) == bad and rn(x=None) == bad
     assert rn(M=0, x=None) == qb.QI21_OK
+    ls = lambda N=512: lib.qi21_linear_swiglu(32, N, 64, p(16), p(16), None, p(16), p(256), 256, None)
+    assert ls(N=384) == bad and ls(N=200) == bad                  # gate/up blocks of 128 need N % 256 == 0
     sw = lambda n=64, g=16: lib.qi21_swiglu(n, p(g) if g else None, p(16), p(16), None)
     assert sw(n=60) == bad and sw(n=-8) == bad and sw(g=None) == bad and sw(g=8) == bad
     assert sw(n=0, g=None) == qb.QI21_OK

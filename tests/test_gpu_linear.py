@@ -58,6 +58,26 @@ def test_linear_shapes(cuda_device, M, N, K, n_out, bias):
     _check(got, x, w, b, what="linear %dx%dx%d/%d" % (M, N, K, n_out))
 
 
+@pytest.mark.parametrize("M,F,K", [(200, 384, 136), (4096, 1536, 512)])
+def test_linear_swiglu(cuda_device, M, F, K):
+    """silu(x W_g^T + b_g) * (x W_u^T + b_u) from one launch, weights given to
+    the GPU in the alternating-block layout, against the float64 oracle with
+    the plain [gate; up] layout."""
+    x, w, b = _draw(M, 2 * F, K, seed=M + F)
+    dev = cuda_device
+    got = qi.linear_swiglu(x.to(dev), qi.interleave_gate_up(w).to(dev), qi.interleave_gate_up(b).to(dev)).cpu()
+    xf, wf, bf = W.as_f64(x), W.as_f64(w), W.as_f64(b)
+    gu = O.linear(xf, wf, bf)
+    g, u = gu[:, :F], gu[:, F:]
+    ref = O.silu(g) * u
+    # one bf16 rounding of the result plus the fp32 accumulation of g and u
+    # carried through silu(g) * u (|d silu / dg| <= 1.1)
+    acc = 2.0 ** -16 * (np.abs(xf) @ np.abs(wf).T)
+    bound = 2.0 ** -8 * np.abs(ref) + 1.1 * np.abs(u) * acc[:, :F] + np.abs(O.silu(g)) * acc[:, F:]
+    err = np.abs(got.double().numpy() - ref)
+    assert np.all(err <= bound + 1e-6), float(np.max(err - bound))
+
+
 def test_linear_target_qkv_full_size_sampled(cuda_device):
     """The t2i cached step's fused Q/K/V projection: 4096 target tokens,
     hidden 3072 = 24 heads x 128, N = 3 x 3072; sampled rows against the oracle."""
