@@ -61,3 +61,37 @@ def test_bench_flops_match_oracle_pair_count(name):
     bh = cfg["B"] * cfg["H"]
     assert full == 4 * 128 * O.allowed_pairs(kv_end) * bh
     assert cached == (0 if orig else 4 * 128 * T * (P + T) * bh)
+
+
+def _worker_one_leaves(rank, world, port, out):
+    """Rank 1 leaves between steps (no collective in flight); rank 0's next
+    collective must end with an error within the short timeout, not hang."""
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    dev = torch.device("cpu")
+    bench.max_over_ranks(1.0, world, dev)  # one good step together
+    if rank == 1:
+        out[rank] = "left"
+        os._exit(0)
+    t0 = time.monotonic()
+    try:
+        bench.max_over_ranks(2.0, world, dev)
+        out[rank] = "no error"
+    except Exception:
+        out[rank] = "error after %.1f s" % (time.monotonic() - t0)
+    os._exit(0)
+
+
+def test_rank_that_leaves_is_detected_gloo():
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker_one_leaves, args=(world, port, out), nprocs=world, start_method="spawn",
+                       join=True)
+    assert out[1] == "left"
+    assert out[0].startswith("error after"), out[0]
+    assert float(out[0].split()[2]) < 30.0
