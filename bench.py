@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch, from the ncu capture summarised in
 # profiles/attn_tc_t2i.md (mean of the full-step and cached-step launches).  Valid only
 # for the kernel source it was taken on: a different attn_tc.cu reports null.
-NCU_TRAFFIC = {"attn_tc_source_sha256": "58135c3ca9e5b02d",
-               "bytes_per_launch": {"t2i": (145.19e6 + 134.06e6) / 2}}
+NCU_TRAFFIC = {"attn_tc_source_sha256": "2174bfda04694bc4",
+               "bytes_per_launch": {"t2i": (147.90e6 + 132.26e6) / 2}}
 
 
 def ncu_traffic(name):
