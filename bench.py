@@ -551,7 +551,8 @@ def run_ours(args, world, rank, local):
     full_tf = full_flops * args.steps / (full_ms * 1e-3) / 1e12
     cached_tf = cached_flops * args.steps / (cached_ms * 1e-3) / 1e12 if cached_flops else None
 
-    budget = 0.0 if args.no_cpu_baseline else args.cpu_budget
+    # the oracle baseline runs on rank 0 of a one-GPU run only
+    budget = 0.0 if (args.no_cpu_baseline or world > 1) else args.cpu_budget
     cpu = None
     if budget > 0:
         f, s, heads = oracle_sample(name, budget)
