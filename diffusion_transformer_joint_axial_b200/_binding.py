@@ -24,12 +24,18 @@ HEAD_DIM = 128
 MAX_SEGMENTS = 128
 WORKSPACE_HEADER_BYTES = 256
 
-EXPORTED = ("qi21_rope_positions", "qi21_attn_full_workspace_size", "qi21_attn_full",
-            "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_workspace_status",
-            "qi21_selftest_wait_timeout", "qi21_status_string", "qi21_last_error",
-            "qi21_launch_count", "qi21_time_next_attention", "qi21_attn_cached_noalloc", "qi21_selftest_exp2",
-            "qi21_attn_full_qknorm", "qi21_attn_cached_qknorm", "qi21_linear", "qi21_rope_positions_original",
-            "qi21_linear_residual", "qi21_rmsnorm", "qi21_swiglu", "qi21_linear_swiglu")
+EXPORTED = (
+    # positions and the attention steps
+    "qi21_rope_positions", "qi21_rope_positions_original",
+    "qi21_attn_full_workspace_size", "qi21_attn_full", "qi21_attn_full_qknorm",
+    "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_attn_cached_qknorm",
+    "qi21_attn_cached_noalloc",
+    # projections and the rest of a block of the denoising loop
+    "qi21_linear", "qi21_linear_residual", "qi21_linear_swiglu", "qi21_rmsnorm", "qi21_swiglu",
+    # status, errors, counters, timing and self-tests
+    "qi21_workspace_status", "qi21_status_string", "qi21_last_error", "qi21_launch_count",
+    "qi21_time_next_attention", "qi21_selftest_wait_timeout", "qi21_selftest_exp2",
+)
 
 
 class QI21Error(RuntimeError):
