@@ -234,6 +234,7 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   rp.k_dst1 = cache ? ws_k : nullptr;
   rp.v_dst0 = cache ? v_cache : nullptr;
   rp.table = table;
+  rp.table_half = dt == QI21_BF16 ? 1 : 0;
   rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;
@@ -309,6 +310,7 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   rp.split = T;
   rp.k_dst0 = ws_k;
   rp.table = table;
+  rp.table_half = dt == QI21_BF16 ? 1 : 0;
   rp.unit_counter = &reinterpret_cast<WsHeader*>(ws)->unit_counter;
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;

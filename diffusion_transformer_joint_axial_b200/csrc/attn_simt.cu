@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     float y0 = 0.f, y1 = 0.f;
     if (row < a.Lq) {
       const float* src = q + (b * a.Lq + row) * tok_stride + h * kHeadDim + 2 * m;
-      const float2 cs = a.table[row * kPairs + m];
+      const float2 cs = static_cast<const float2*>(a.table)[row * kPairs + m];
       float x0 = src[0], x1 = src[1];
       if (norm) {
         x0 *= s_rs[r] * a.q_norm_w[2 * m];

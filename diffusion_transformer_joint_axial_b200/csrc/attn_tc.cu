@@ -37,6 +37,7 @@
 // Online softmax uses a lazy rescale: O and l are rescaled only when a row
 // maximum grows by more than 2^8, which keeps every P <= 256.
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "qi21_device.cuh"
@@ -87,7 +88,7 @@ struct Params {
   int32_t B, H, Lq, n0, n1;
   int32_t nqp;        // query-tile pairs per (batch, head)
   int32_t num_units;  // B * H * nqp
-  const float2* table;
+  const uint4* table;  // per token 16 x (4 x half2 (cos, sin)): one 16-byte load per 8 dims
   const int32_t* kv_end;
   __nv_bfloat16* o;
   uint32_t* status;
@@ -186,7 +187,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
 // the row's mean square (fp32, from the bf16 values), then each adjacent pair
 // (2m, 2m+1) scaled by rsqrt(mean square + eps) and the weight and rotated by
 // the token's (cos, sin), rounded once to bf16.
-__device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const float4* cs, int t,
+__device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const uint4* cs, int t,
                                                   const float* wn, float eps) {
   float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll 4
@@ -207,19 +208,18 @@ __device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const float4* c
     const int half = c >> 3, cc = c & 7;
     uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
     uint4 x = *ptr;
-    const float4 r01 = __ldg(cs + 2 * c);
-    const float4 r23 = __ldg(cs + 2 * c + 1);
     const float4 w0 = *reinterpret_cast<const float4*>(wn + 8 * c);
     const float4 w1 = *reinterpret_cast<const float4*>(wn + 8 * c + 4);
     const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    const float cv[4] = {r01.x, r01.z, r23.x, r23.z};
-    const float sv[4] = {r01.y, r01.w, r23.y, r23.w};
+    const uint4 tb = __ldg(cs + c);  // the chunk's four (cos, sin) pairs
+    const __half2* tc = reinterpret_cast<const __half2*>(&tb);
     uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 v = unpack_bf16x2(w[e]);
+      const float2 r = __half22float2(tc[e]);  // (cos, sin)
       const float x0 = v.x * rs * wv[2 * e], x1 = v.y * rs * wv[2 * e + 1];
-      w[e] = pack_bf16x2(fmaf(x0, cv[e], -x1 * sv[e]), fmaf(x0, sv[e], x1 * cv[e]));
+      w[e] = pack_bf16x2(fmaf(x0, r.x, -x1 * r.y), fmaf(x0, r.y, x1 * r.x));
     }
     *ptr = x;
   }
@@ -652,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t par = qv & 1u;  // unit parity of this tile's l buffer
       ++qv;
       if (valid) {
-        const float4* cs = reinterpret_cast<const float4*>(p.table + (size_t)row * kPairs);
+        const uint4* cs = p.table + (size_t)row * 16;
         uint8_t* qrow = S.q[s] + t * 128;
         if (p.q_norm_w == nullptr) {
 #pragma unroll 4
@@ -660,17 +660,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int half = c >> 3, cc = c & 7;
             uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
             uint4 x = *ptr;
-            const float4 r01 = __ldg(cs + 2 * c);
-            const float4 r23 = __ldg(cs + 2 * c + 1);
+            const uint4 tb = __ldg(cs + c);  // the chunk's four (cos, sin) pairs
+            const __half2* tc = reinterpret_cast<const __half2*>(&tb);
             uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-            float2 xv = unpack_bf16x2(w[0]);
-            w[0] = pack_bf16x2(fmaf(xv.x, r01.x, -xv.y * r01.y), fmaf(xv.x, r01.y, xv.y * r01.x));
-            xv = unpack_bf16x2(w[1]);
-            w[1] = pack_bf16x2(fmaf(xv.x, r01.z, -xv.y * r01.w), fmaf(xv.x, r01.w, xv.y * r01.z));
-            xv = unpack_bf16x2(w[2]);
-            w[2] = pack_bf16x2(fmaf(xv.x, r23.x, -xv.y * r23.y), fmaf(xv.x, r23.y, xv.y * r23.x));
-            xv = unpack_bf16x2(w[3]);
-            w[3] = pack_bf16x2(fmaf(xv.x, r23.z, -xv.y * r23.w), fmaf(xv.x, r23.w, xv.y * r23.z));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xv = unpack_bf16x2(w[e]);
+              const float2 r = __half22float2(tc[e]);  // (cos, sin) of pair 4c + e
+              w[e] = pack_bf16x2(fmaf(xv.x, r.x, -xv.y * r.y), fmaf(xv.x, r.y, xv.y * r.x));
+            }
             *ptr = x;
           }
         } else {
@@ -836,7 +834,7 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.n1 = (int32_t)a.k1.n;
   p.nqp = (int32_t)((a.Lq + 2 * tc::BM - 1) / (2 * tc::BM));
   p.num_units = a.B * a.H * p.nqp;
-  p.table = a.table;
+  p.table = static_cast<const uint4*>(a.table);
   p.kv_end = a.kv_end;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.status = a.status;

@@ -58,7 +58,8 @@ struct RopePrepParams {
   void* k_dst0;    // head-major [B, H, split, 128]
   void* k_dst1;    // head-major [B, H, Lk - split, 128] (or null when split == Lk)
   void* v_dst0;    // head-major [B, H, split, 128] copy of V, or null
-  float2* table;   // [Lk][64] (cos, sin) of every token, or null
+  void* table;     // [Lk][64] (cos, sin) of every token, or null: float2, or half2 when table_half
+  int32_t table_half;
   uint32_t* unit_counter;  // zeroed here for the attention launch that follows, or null
   Omega omega;
   const float* k_norm_w;   // [128] QK-RMSNorm weight of K, or null (no norm)
@@ -81,7 +82,7 @@ struct AttnArgs {
   int32_t B, H;
   int64_t Lq;
   const void* q;          // token-major [B, Lq, H, 128] (not rotated)
-  const float2* table;    // [Lq][64] cos/sin of the query rows
+  const void* table;      // [Lq][64] cos/sin of the query rows: half2 (bf16 path) or float2 (fp32)
   const int32_t* kv_end;  // [Lq] or null
   KvSource k0, k1;        // rotated keys
   KvSource v0, v1;        // values
