@@ -43,3 +43,19 @@ def test_seeded_inputs_are_deterministic():
     p1, _ = W.denoise_model(1, 16, 1, 2, seed=5, dtype="f32")
     p2, _ = W.denoise_model(1, 16, 1, 2, seed=5, dtype="f32")
     assert torch.equal(p1["blocks"][0]["w_gu"], p2["blocks"][0]["w_gu"])
+
+
+def test_fp16_rotation_table_error_bound():
+    """The bf16 path rotates its queries with (cos, sin) rounded to fp16; over
+    every position of every workload they stay within 2.4e-4 (2^-12) of the
+    float64 values, a tenth of the bf16 rounding of a rotated query."""
+    import oracle as O
+    worst = 0.0
+    for name, cfg in W.WORKLOADS.items():
+        fn = O.positions_original if cfg.get("original") else O.positions
+        pos, _ = fn(cfg["segments"])
+        ang = O.rope_angles(pos)
+        for f in (np.cos, np.sin):
+            exact = f(ang)
+            worst = max(worst, float(np.max(np.abs(exact.astype(np.float16).astype(np.float64) - exact))))
+    assert worst <= 2.0 ** -12, worst
