@@ -346,8 +346,10 @@ def _split(y, parts):
     return [y[..., i * n:(i + 1) * n] for i in range(parts)]
 
 
-def _block_attention(h, blk, eps, attend):
-    """h + (attend(q, k, v) W_o^T + b_o) with q, k, v from RMSNorm(h)."""
+def block_attention(h, blk, eps, attend):
+    """Attention half of a block (overview card 4A): h + (attend(q, k, v) W_o^T + b_o),
+    with q, k, v the three thirds of RMSNorm(h; norm1) W_qkv^T + b_qkv, each
+    split into 128-wide heads."""
     B, L, D = h.shape
     a = rms_norm(h, blk["norm1"], eps)
     q, k, v = (t.reshape(B, L, D // HEAD_DIM, HEAD_DIM) for t in _split(linear(a, blk["w_qkv"], blk["b_qkv"]), 3))
@@ -355,11 +357,31 @@ def _block_attention(h, blk, eps, attend):
     return h + linear(o.reshape(B, L, D), blk["w_o"], blk["b_o"])
 
 
-def _block_ffn(h, blk, eps):
-    """h + (silu(g) * u) W_down^T + b_down with [g | u] from RMSNorm(h)."""
+def block_ffn(h, blk, eps):
+    """Feed-forward half of a block (card 5A, SwiGLU): h + (silu(g) * u) W_down^T
+    + b_down, with the gate g first and the up branch u second in
+    [g | u] = RMSNorm(h; norm2) W_gu^T + b_gu."""
     a = rms_norm(h, blk["norm2"], eps)
     g, u = _split(linear(a, blk["w_gu"], blk["b_gu"]), 2)
     return h + linear(silu(g) * u, blk["w_down"], blk["b_down"])
+
+
+def block(h, blk, eps, attend):
+    """One block: the attention half, then the feed-forward half (cards 4A, 5A)."""
+    return block_ffn(block_attention(h, blk, eps, attend), blk, eps)
+
+
+def embed(x, params, step):
+    """Target latents to hidden states: x W_in^T + b_in[step] (card 1A: the
+    latent patches enter the DiT through a linear map; the per-step bias
+    stands for the step's conditioning of the target tokens)."""
+    return linear(x, params["w_in"], params["b_in"][step])
+
+
+def velocity(h_t, params, eps):
+    """Velocity head (card 6B): RMSNorm(h_t; norm_out) W_v^T + b_v on the
+    target tokens."""
+    return linear(rms_norm(h_t, params["norm_out"], eps), params["w_v"], params["b_v"])
 
 
 def denoise(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
@@ -380,7 +402,7 @@ def denoise(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
     prefix_h = np.asarray(prefix_h, dtype=np.float64)
     caches = [None] * len(params["blocks"])
     for step in range(len(sigmas) - 1):
-        h_t = linear(x, params["w_in"], params["b_in"][step])
+        h_t = embed(x, params, step)
         if step == 0 or not cached:
             h = np.concatenate([prefix_h, h_t], axis=1)
             for i, blk in enumerate(params["blocks"]):
@@ -388,16 +410,15 @@ def denoise(x0, prefix_h, params, segments, sigmas, cached=True, eps=1e-6):
                     if cached:
                         caches[i] = prefix_cache(k, v, pos, P)
                     return attn_full(q, k, v, pos, kv_end)
-                h = _block_ffn(_block_attention(h, blk, eps, attend), blk, eps)
+                h = block(h, blk, eps, attend)
             h_t = h[:, P:]
         else:
             h = h_t
             for i, blk in enumerate(params["blocks"]):
                 attend = lambda q, k, v, i=i: attn_cached(q, k, v, pos[P:], caches[i][0], caches[i][1])
-                h = _block_ffn(_block_attention(h, blk, eps, attend), blk, eps)
+                h = block(h, blk, eps, attend)
             h_t = h
-        vel = linear(rms_norm(h_t, params["norm_out"], eps), params["w_v"], params["b_v"])
-        x = x + (sigmas[step + 1] - sigmas[step]) * vel
+        x = x + (sigmas[step + 1] - sigmas[step]) * velocity(h_t, params, eps)
     return x
 
 

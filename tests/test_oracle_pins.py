@@ -375,13 +375,146 @@ def check_denoise_euler_closed_form(O):
     assert np.max(np.abs(x - (x0 - c))) < 1e-14
 
 
+# Pins of the loop's stages, each against a closed form that fixes its
+# composition (overview cards 4A, 5A, 6B): with identity-structured weights
+# every stage reduces to a few scalar formulas, evaluated here with plain
+# Python loops and math.exp / math.sqrt.
+
+def _rms_scalar(row, w, eps):
+    r = 1.0 / math.sqrt(sum(x * x for x in row) / len(row) + eps)
+    return [x * r * wi for x, wi in zip(row, w)]
+
+
+def _silu_scalar(x):
+    return x / (1.0 + math.exp(-x))
+
+
+def _single_key_block(D=128, seed=31):
+    rng = np.random.default_rng(seed)
+    h = rng.standard_normal((1, 1, D)) * 3.0 + 0.5
+    blk = dict(norm1=1 + 0.1 * rng.standard_normal(D),
+               w_qkv=np.concatenate([rng.standard_normal((2 * D, D)), np.eye(D)]),  # value third = I
+               b_qkv=np.zeros(3 * D), w_o=np.eye(D), b_o=0.05 * rng.standard_normal(D),
+               norm2=1 + 0.1 * rng.standard_normal(D),
+               w_gu=np.concatenate([np.eye(D), 2.0 * np.eye(D)]),  # gate = a, up = 2a
+               b_gu=np.zeros(2 * D), w_down=np.eye(D), b_down=0.05 * rng.standard_normal(D))
+    return h, blk
+
+
+def _attend_first_text_token(O):
+    pos, kv = O.positions([W.text(1)])
+    return lambda q, k, v: O.attn_full(q, k, v, pos, kv)
+
+
+def _expect_attention_half(h, blk, eps=1e-6):
+    """Token 0 of the text sees only itself (card 3C), so its attention
+    weights are [1] and the output is its own V = RMSNorm(h; norm1);
+    W_o = I: h + RMSNorm(h; norm1) + b_o."""
+    a = _rms_scalar(h, blk["norm1"], eps)
+    return [x + y + b for x, y, b in zip(h, a, blk["b_o"])]
+
+
+def _expect_ffn_half(h, blk, eps=1e-6):
+    """[g | u] = [a | 2a] with a = RMSNorm(h; norm2), W_down = I:
+    h + silu(a) * 2a + b_down (card 5A: the gate passes through SiLU)."""
+    a = _rms_scalar(h, blk["norm2"], eps)
+    return [x + _silu_scalar(ai) * 2.0 * ai + b for x, ai, b in zip(h, a, blk["b_down"])]
+
+
+def check_block_attention_single_key(O):
+    h, blk = _single_key_block()
+    got = O.block_attention(h, blk, 1e-6, _attend_first_text_token(O))
+    exp = np.array(_expect_attention_half(list(h[0, 0]), blk))
+    assert np.max(np.abs(got[0, 0] - exp)) < 1e-12
+
+
+def check_block_ffn_closed_form(O):
+    h, blk = _single_key_block(seed=32)
+    got = O.block_ffn(h, blk, 1e-6)
+    exp = np.array(_expect_ffn_half(list(h[0, 0]), blk))
+    assert np.max(np.abs(got[0, 0] - exp)) < 1e-12
+
+
+def check_block_order(O):
+    """A block is the attention half, then the feed-forward half on its
+    result (cards 4A then 5A)."""
+    h, blk = _single_key_block(seed=33)
+    got = O.block(h, blk, 1e-6, _attend_first_text_token(O))
+    exp = np.array(_expect_ffn_half(_expect_attention_half(list(h[0, 0]), blk), blk))
+    assert np.max(np.abs(got[0, 0] - exp)) < 1e-12
+
+
+def check_velocity_closed_form(O):
+    """Card 6B: the velocity is the RMS-normalised target state through W_v.
+    A row of constant c normalises to c / sqrt(c^2 + eps) in every dim; with
+    W_v = I the velocity is that times norm_out, plus b_v."""
+    rng = np.random.default_rng(34)
+    D, eps = 128, 1e-6
+    c = np.array([0.5, -3.0, 7.0])
+    h = np.repeat(c[None, :, None], D, axis=2)
+    params = dict(norm_out=1 + 0.1 * rng.standard_normal(D), w_v=np.eye(D), b_v=0.1 * rng.standard_normal(D))
+    got = O.velocity(h, params, eps)
+    for t, ct in enumerate(c):
+        exp = [ct / math.sqrt(ct * ct + eps) * w + b for w, b in zip(params["norm_out"], params["b_v"])]
+        assert np.max(np.abs(got[0, t] - np.array(exp))) < 1e-13
+
+
+def check_denoise_explicit_one_step(O):
+    """One Euler step of a one-block model over a text token and a 1x1
+    target, every stage written as explicit scalar loops: embedding (card
+    1A), RMSNorm -> Q/K/V -> block-causal softmax attention -> W_o ->
+    residual (card 4A; text token 0 sees itself, the target sees both),
+    RMSNorm -> SwiGLU -> W_down -> residual (card 5A), velocity from the
+    RMS-normalised target state and x1 = x0 + (sigma1 - sigma0) v (card
+    6B).  The rotation uses the oracle's own rope (pinned above by the
+    close reading's polar construction)."""
+    rng = np.random.default_rng(35)
+    D, C, F, eps = 128, 4, 384, 1e-6
+    r = lambda *s, sc=1.0: sc * rng.standard_normal(s)
+    blk = dict(norm1=1 + 0.1 * r(D), w_qkv=r(3 * D, D, sc=D ** -0.5), b_qkv=r(3 * D, sc=0.1),
+               w_o=r(D, D, sc=D ** -0.5), b_o=r(D, sc=0.1), norm2=1 + 0.1 * r(D),
+               w_gu=r(2 * F, D, sc=D ** -0.5), b_gu=r(2 * F, sc=0.1), w_down=r(D, F, sc=F ** -0.5),
+               b_down=r(D, sc=0.1))
+    params = dict(w_in=r(D, C, sc=C ** -0.5), b_in=r(1, D, sc=0.5), blocks=[blk], norm_out=1 + 0.1 * r(D),
+                  w_v=r(C, D, sc=D ** -0.5), b_v=r(C, sc=0.1))
+    x0, ph = r(1, 1, C), r(1, 1, D)
+    segs = [W.text(1), W.image(1, 1, 0)]
+    sig = [1.0, 0.4]
+    got = O.denoise(x0, ph, params, segs, sig, cached=True, eps=eps)
+
+    mv = lambda w, x, b: [sum(w[n][kk] * x[kk] for kk in range(len(x))) + b[n] for n in range(len(w))]
+    h = [list(ph[0, 0]), mv(params["w_in"], list(x0[0, 0]), params["b_in"][0])]
+    qkv = [mv(blk["w_qkv"], _rms_scalar(row, blk["norm1"], eps), blk["b_qkv"]) for row in h]
+    pos = np.array([[0, 0, 0], [0, -1, -1]])  # text 0; 1x1 image centred at -(1 - 0) = -1
+    q = O.rope(np.array([t[:D] for t in qkv]), pos)
+    k = O.rope(np.array([t[D:2 * D] for t in qkv]), pos)
+    v = [t[2 * D:] for t in qkv]
+    h1 = []
+    for i in range(2):
+        s = [sum(q[i][d] * k[j][d] for d in range(D)) / math.sqrt(D) for j in range(i + 1)]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        o = [sum(e[j] * v[j][d] for j in range(i + 1)) / sum(e) for d in range(D)]
+        h1.append([a + b for a, b in zip(h[i], mv(blk["w_o"], o, blk["b_o"]))])
+    h2 = []
+    for row in h1:
+        gu = mv(blk["w_gu"], _rms_scalar(row, blk["norm2"], eps), blk["b_gu"])
+        mid = [_silu_scalar(gu[f]) * gu[F + f] for f in range(F)]
+        h2.append([a + b for a, b in zip(row, mv(blk["w_down"], mid, blk["b_down"]))])
+    vel = mv(params["w_v"], _rms_scalar(h2[1], params["norm_out"], eps), params["b_v"])
+    exp = [x + (sig[1] - sig[0]) * vv for x, vv in zip(x0[0, 0], vel)]
+    assert np.max(np.abs(got[0, 0] - np.array(exp))) < 1e-11
+
+
 CHECKS = [check_page_example_h4, check_centring_neg_pos_tables, check_text_and_frames,
           check_prompt_length_invariance, check_block_causal_rule, check_prefix_never_sees_target,
           check_bands, check_rope_vs_polar, check_rope_invariants, check_attention_brute_force,
           check_attention_closed_forms, check_attention_vs_sdpa, check_prefix_invariance,
           check_cached_equals_full, check_rms_norm_vs_torch, check_rms_norm_closed_forms,
           check_linear_brute_force, check_linear_special_cases, check_original_text_offset,
-          check_silu_vs_torch, check_denoise_cache_reuse, check_denoise_euler_closed_form]
+          check_silu_vs_torch, check_denoise_cache_reuse, check_denoise_euler_closed_form,
+          check_block_attention_single_key, check_block_ffn_closed_form, check_block_order,
+          check_velocity_closed_form, check_denoise_explicit_one_step]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda f: f.__name__)
@@ -532,6 +665,45 @@ def _denoise_stale_target(x0, prefix_h, params, segments, sigmas, cached=True, e
     return x + (OM.denoise(x, prefix_h, params, segments, sigmas[1:], False, eps) - x) * 0.5
 
 
+_ORIG_BLOCK_ATTENTION, _ORIG_BLOCK_FFN = OM.block_attention, OM.block_ffn
+
+
+def _ffn_gate_up_swapped(h, blk, eps):
+    a = OM.rms_norm(h, blk["norm2"], eps)
+    g, u = OM._split(OM.linear(a, blk["w_gu"], blk["b_gu"]), 2)
+    return h + OM.linear(OM.silu(u) * g, blk["w_down"], blk["b_down"])
+
+
+def _ffn_norm2_dropped(h, blk, eps):
+    g, u = OM._split(OM.linear(h, blk["w_gu"], blk["b_gu"]), 2)
+    return h + OM.linear(OM.silu(g) * u, blk["w_down"], blk["b_down"])
+
+
+def _attn_residual_dropped(h, blk, eps, attend):
+    B, L, D = h.shape
+    a = OM.rms_norm(h, blk["norm1"], eps)
+    q, k, v = (t.reshape(B, L, D // 128, 128) for t in OM._split(OM.linear(a, blk["w_qkv"], blk["b_qkv"]), 3))
+    return OM.linear(attend(q, k, v).reshape(B, L, D), blk["w_o"], blk["b_o"])
+
+
+def _block_order_swapped(h, blk, eps, attend):
+    return _ORIG_BLOCK_ATTENTION(_ORIG_BLOCK_FFN(h, blk, eps), blk, eps, attend)
+
+
+def _velocity_norm_dropped(h_t, params, eps):
+    return OM.linear(h_t, params["w_v"], params["b_v"])
+
+
+def _embed_bias_dropped(x, params, step):
+    return OM.linear(x, params["w_in"])
+
+
+# Stages that ``denoise`` looks up in the oracle module at call time: these
+# mutants are also planted in the module itself while the pins run, so that
+# the loop uses them.
+STAGE_MUTANTS = {"ffn_gate_up_swapped", "ffn_norm2_dropped", "attn_residual_dropped",
+                 "block_order_swapped", "velocity_norm_dropped", "embed_bias_dropped"}
+
 MUTANTS = {
     "rope_sign": dict(rope=_rope_sign_flipped),
     "band_denominator_128": dict(rope=_rope_with(_angles_global_denominator),
@@ -550,12 +722,21 @@ MUTANTS = {
     "silu_as_sigmoid": dict(silu=_silu_as_sigmoid),
     "euler_step_sign": dict(denoise=_denoise_step_sign),
     "cache_not_reused_faithfully": dict(denoise=_denoise_stale_target),
+    "ffn_gate_up_swapped": dict(block_ffn=_ffn_gate_up_swapped),
+    "ffn_norm2_dropped": dict(block_ffn=_ffn_norm2_dropped),
+    "attn_residual_dropped": dict(block_attention=_attn_residual_dropped),
+    "block_order_swapped": dict(block=_block_order_swapped),
+    "velocity_norm_dropped": dict(velocity=_velocity_norm_dropped),
+    "embed_bias_dropped": dict(embed=_embed_bias_dropped),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutants_are_caught(name):
+def test_mutants_are_caught(name, monkeypatch):
     ns = _mutant(**MUTANTS[name])
+    if name in STAGE_MUTANTS:
+        for k, fn in MUTANTS[name].items():
+            monkeypatch.setattr(OM, k, fn)
     failed = []
     for check in CHECKS:
         try:
