@@ -38,20 +38,25 @@ from diffusion_transformer_joint_axial_b200 import workloads as W  # noqa: E402
 METRIC = "joint-attn TFLOP/s (full step & prefix-cached step), % of B200 BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per attention launch, from the ncu capture summarised in
-# profiles/attn_tc_t2i.md (mean of the full-step and cached-step launches).  Valid only
-# for the kernel source it was taken on: a different attn_tc.cu reports null.
-NCU_TRAFFIC = {"attn_tc_source_sha256": "2174bfda04694bc4",
-               "bytes_per_launch": {"t2i": (147.90e6 + 132.26e6) / 2}}
+# DRAM bytes (read + write) per attention call -- the rotation/cache
+# pre-pass plus the attention kernel -- from one ncu capture of each kernel
+# (dram__bytes_read.sum + dram__bytes_write.sum), per workload.  Valid only for
+# the kernel sources they were taken on: any other source reports null.
+NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_call": {}}
+
+
+def kernel_sources_digest():
+    h = hashlib.sha256()
+    for name in ("attn_tc.cu", "prep_kernels.cu"):
+        with open(os.path.join(ROOT, "diffusion_transformer_joint_axial_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(name):
-    src = os.path.join(ROOT, "diffusion_transformer_joint_axial_b200", "csrc", "attn_tc.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    if digest != NCU_TRAFFIC["attn_tc_source_sha256"]:
+    if NCU_TRAFFIC["sources_sha256"] != kernel_sources_digest():
         return None
-    return NCU_TRAFFIC["bytes_per_launch"].get(name)
+    return NCU_TRAFFIC["bytes_per_call"].get(name)
 
 
 # ------------------------------------------------------------------ helpers --
@@ -89,48 +94,70 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """SM clock and clock-event reasons sampled on a background thread (NVML)
+    while the timed regions run; falls back to ``nvidia-smi -lms`` polling.
+    Only samples taken between ``start()`` and ``pause()`` count, so several
+    short timed regions add up to one record."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index):
-        self.proc = None
+    def __init__(self, device):
+        import threading
+        self.sm, self.reasons, self.power = [], set(), []
+        self.sm_max = None
+        self.active = threading.Event()
+        self.done = threading.Event()
+        self.handle = None
+        self.error = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "20"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            # nvidia-smi takes a moment to start: wait for its first sample
-            # (taken before the timed region, not counted) so that sampling
-            # covers the whole timed region.
-            self.proc.stdout.readline()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                         props.pci_device_id)
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except pynvml.NVMLError:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.nvml = pynvml
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: nothing recorded, and the record says why
+            self.error = "NVML unavailable (%s)" % type(e).__name__
+            return
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def _loop(self):
+        nv = self.nvml
+        while not self.done.is_set():
+            if self.active.wait(0.05):
+                try:
+                    self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    for name, bit in self.REASONS:
+                        if r & bit:
+                            self.reasons.add(name)
+                    self.power.append(nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0)
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+    def start(self):
+        self.active.set()
+
+    def pause(self):
+        self.active.clear()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                sm.append(float(f[0]))
-                smax.append(float(f[1]))
-            except ValueError:
-                continue
-            for n, val in zip(names, f[4:8]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self.pause()
+        self.done.set()
+        if self.error:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error], "samples": 0}
+        self.thread.join(timeout=5)
+        return {"sm_mhz": statistics.median(self.sm) if self.sm else None, "sm_max_mhz": self.sm_max,
+                "reasons": sorted(self.reasons), "samples": len(self.sm),
+                "power_w_max": max(self.power) if self.power else None, "source": "NVML, 2 ms polling"}
 
 
 def dist_setup(args):
@@ -169,10 +196,15 @@ def barrier(world):
 
 # ---------------------------------------------------------------- CPU oracle --
 
-def oracle_sample(name, budget_s):
-    """Times the float64 oracle on a bounded sample of the workload: whole
-    heads of the full step and of one cached step, until ``budget_s`` passes.
-    Returns (flops, seconds, heads done)."""
+ORACLE_ROWS = 512  # query rows per oracle piece
+
+
+def oracle_sample(name, budget_s, max_pieces=None):
+    """Times the float64 oracle on a bounded sample of the workload: pieces of
+    ORACLE_ROWS query rows of one head, one piece of the full step (rows taken
+    in turn along the sequence, so text, reference and target rows all come
+    up) plus one piece of the cached step, until ``budget_s`` passes (at least
+    one piece).  Returns (algorithmic flops of the rows done, seconds, pieces)."""
     import oracle as O
     cfg = W.WORKLOADS[name]
     L, P, T = W.sizes(name)
@@ -180,19 +212,26 @@ def oracle_sample(name, budget_s):
     qf, kf, vf = W.as_f64(q), W.as_f64(k), W.as_f64(v)
     orig = cfg.get("original", False)
     pos, kv_end = (O.positions_original if orig else O.positions)(cfg["segments"])
-    full1, cached1 = (x / (cfg["B"] * cfg["H"]) for x in step_flops(name))
-    flops, heads = 0.0, 0
+    kv_end = np.asarray(kv_end, dtype=np.int64)
+    kc = vc = None
+    flops, pieces = 0.0, 0
     t0 = time.perf_counter()
     while True:
-        O.attn_full(qf, kf, vf, pos, kv_end)
+        r0 = (pieces * ORACLE_ROWS) % L
+        rows = np.arange(r0, min(L, r0 + ORACLE_ROWS))
+        O.attn_full(qf, kf, vf, pos, kv_end, rows=rows)
+        flops += 4.0 * 128 * float(kv_end[rows].sum())
         if not orig:
-            kc, vc = O.prefix_cache(kf, vf, pos, P)
-            O.attn_cached(qf[:, P:], kf[:, P:], vf[:, P:], pos[P:], kc, vc)
-        flops += full1 + cached1
-        heads += 1
+            if kc is None:
+                kc, vc = O.prefix_cache(kf, vf, pos, P)
+            c0 = (pieces * ORACLE_ROWS) % T
+            crows = np.arange(c0, min(T, c0 + ORACLE_ROWS))
+            O.attn_cached(qf[:, P:], kf[:, P:], vf[:, P:], pos[P:], kc, vc, rows=crows)
+            flops += 4.0 * 128 * len(crows) * (P + T)
+        pieces += 1
         dt = time.perf_counter() - t0
-        if dt >= budget_s or heads >= cfg["B"] * cfg["H"]:
-            return flops, dt, heads
+        if dt >= budget_s or (max_pieces is not None and pieces >= max_pieces):
+            return flops, dt, pieces
 
 
 def cpu_cores():
@@ -203,20 +242,23 @@ def cpu_cores():
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the float64 oracle (the only CPU implementation of
+    the method) timed on the host cores, one oracle piece per step, on the
+    headline workload's shapes; rank 0 only."""
     if rank != 0:
         return
-    name = args.workload
+    name = headline_workload(args)
     cfg = W.WORKLOADS[name]
     for _ in range(args.warmup):
-        oracle_sample(name, 0.0)
-    tot_f, tot_s, heads = 0.0, 0.0, 0
+        oracle_sample(name, 0.0, max_pieces=1)
+    tot_f, tot_s, pieces = 0.0, 0.0, 0
     for _ in range(args.steps):
-        f, s, h = oracle_sample(name, 0.0)
-        tot_f, tot_s, heads = tot_f + f, tot_s + s, heads + h
+        f, s, n = oracle_sample(name, 0.0, max_pieces=1)
+        tot_f, tot_s, pieces = tot_f + f, tot_s + s, pieces + n
     value = tot_f / tot_s / 1e12
-    sample = "%d head(s) of the %s full step%s per bench step (float64 oracle, %s)" % (
-        heads // max(1, args.steps), name, "" if cfg.get("original") else " + one cached step",
-        W.DESCRIPTIONS[name])
+    sample = ("per step: %d query rows of one head of the %s full step%s (float64 NumPy oracle); "
+              "TFLOP/s counts the algorithmic work of the rows done" % (
+                  ORACLE_ROWS, name, "" if cfg.get("original") else " + %d rows of its cached step" % ORACLE_ROWS))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -403,22 +445,31 @@ def time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops):
     return out
 
 
-def run_ours(args, world, rank, local):
-    import diffusion_transformer_joint_axial_b200 as qi
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    name = args.workload
+BENCH_WORKLOADS = ("t2i", "edit3", "maxref", "hires", "orig")
+# The largest single-GPU configuration (B=2, 16384 target tokens): the line's headline.
+HEADLINE = "hires"
+
+
+def headline_workload(args):
+    return HEADLINE if args.workload == "all" else args.workload
+
+
+def bench_workload(qi, args, name, world, dev, flush, clocks, headline):
+    """Times ``args.steps`` steps of one workload after ``args.warmup``
+    untimed ones.  A step = positions -> full block-causal step with cache
+    store -> one cached step (the earlier model's layout: positions -> one
+    unmasked full step), each a whole C-ABI call (its rotation/cache pre-pass
+    and its attention kernel) bracketed by CUDA events on the launch stream;
+    L2 is flushed before every step, outside the events.  Returns the record
+    of the workload (times are max over ranks) and, for the headline, the raw
+    numbers the JSON line is made of."""
+    lib = qi.load_library()
     cfg = W.WORKLOADS[name]
-    assert cfg["dtype"] == "bf16", "the bench measures the bf16 workloads"
     B, H = cfg["B"], cfg["H"]
     L, P, T = W.sizes(name)
     segs = cfg["segments"]
     dt = torch.bfloat16
-    # the earlier model's workload: positions with text after the images, one
-    # unmasked full step, nothing cached (its text attends the target)
     orig = cfg.get("original", False)
-
-    # inputs (host, pinned) and device-resident copies
     q, k, v = W.full_inputs(name)
     host = [x.pin_memory() for x in ((q, k, v) if orig else (q, k, v) + tuple(W.cached_inputs(name, 2)))]
     dq, dk, dv = (x.to(dev) for x in host[:3])
@@ -426,18 +477,15 @@ def run_ours(args, world, rank, local):
     kc, vc = (None, None) if orig else qi.alloc_cache(B, H, P, dt, dev)
     o_full = torch.empty_like(dq)
     o_c = None if orig else torch.empty_like(dqt)
-    ws_f = qi.new_workspace(qi.full_workspace_size(B, H, L, P, dt), dev)
+    ws_f = qi.new_workspace(qi.full_workspace_size(B, H, L, 0 if orig else P, dt), dev)
     ws_c = qi.new_workspace(256 if orig else qi.cached_workspace_size(B, H, P, T, dt), dev)
     pos = torch.empty((L, 3), dtype=torch.int32, device=dev)
     kv_end = torch.empty((L,), dtype=torch.int32, device=dev)
     assert pos[P:].data_ptr() % 16 == 0, "target rows of the position table must be 16-byte aligned"
     seg_arr = qi._binding.to_segments(segs)
-    lib = qi.load_library()
     stream = torch.cuda.current_stream(dev)
     sp = qi._binding.ctypes.c_void_p(stream.cuda_stream)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     P_ = qi._binding._ptr
-
     if args.qk_norm:  # the fused QK-RMSNorm variant of both steps
         wq, wk = (w.to(dev) for w in W.qk_norm_weights())
         norm = (P_(wq), P_(wk), qi._binding.ctypes.c_float(W.QK_NORM_EPS))
@@ -445,26 +493,26 @@ def run_ours(args, world, rank, local):
         cached_fn = lambda *a: lib.qi21_attn_cached_qknorm(*a[:12], *norm, *a[12:])
     else:
         full_fn, cached_fn = lib.qi21_attn_full, lib.qi21_attn_cached
-
     positions_fn = lib.qi21_rope_positions_original if orig else lib.qi21_rope_positions
 
-    def one_step(ev=None, qq=dq, kk=dk, vv=dv, qqt=dqt, kkt=dkt, vvt=dvt):
-        positions_fn(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
+    def one_step(ev=None):
         if ev is not None:
-            qi.time_next_attention(ev[0], ev[1])
-        st = full_fn(B, H, L, 0 if orig else P, 0, P_(qq), P_(kk), P_(vv), P_(pos), P_(kv_end), P_(o_full),
+            ev[0].record(stream)
+        st = positions_fn(seg_arr, len(segs), L, P_(pos), P_(kv_end), sp)
+        assert st == 0, lib.qi21_last_error()
+        if ev is not None:
+            ev[1].record(stream)
+        st = full_fn(B, H, L, 0 if orig else P, 0, P_(dq), P_(dk), P_(dv), P_(pos), P_(kv_end), P_(o_full),
                      P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
         assert st == 0, lib.qi21_last_error()
-        if orig:
-            if ev is not None:  # no cached step: an empty interval keeps the bookkeeping
-                ev[2].record(stream)
-                ev[3].record(stream)
-            return
         if ev is not None:
-            qi.time_next_attention(ev[2], ev[3])
-        st = cached_fn(B, H, P, T, 0, P_(qqt), P_(kkt), P_(vvt), P_(pos[P:]), P_(kc), P_(vc),
-                       P_(o_c), P_(ws_c), ws_c.numel(), sp)
-        assert st == 0, lib.qi21_last_error()
+            ev[2].record(stream)
+        if not orig:
+            st = cached_fn(B, H, P, T, 0, P_(dqt), P_(dkt), P_(dvt), P_(pos[P:]), P_(kc), P_(vc),
+                           P_(o_c), P_(ws_c), ws_c.numel(), sp)
+            assert st == 0, lib.qi21_last_error()
+        if ev is not None:
+            ev[3].record(stream)
 
     full_flops, cached_flops = step_flops(name)
     for _ in range(args.warmup):
@@ -472,135 +520,171 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
 
-    # ---- device-resident timing
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    evs = [(mk(), mk(), mk(), mk(), mk(), mk()) for _ in range(args.steps)]
+    evs = [(mk(), mk(), mk(), mk()) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
     n0 = qi.launch_count()
-    for i in range(args.steps):
+    for e in evs:
         flush.zero_()
-        e = evs[i]
-        e[4].record(stream)
-        one_step(ev=e)
-        e[5].record(stream)
+        one_step(e)
     torch.cuda.synchronize()
+    if clocks:
+        clocks.pause()
     barrier(world)
     launches = qi.launch_count() - n0
-    clk = clocks.stop() if clocks else None
-    step_ms = sum(e[4].elapsed_time(e[5]) for e in evs)
-    full_each = [e[0].elapsed_time(e[1]) for e in evs]
-    cached_each = [e[2].elapsed_time(e[3]) for e in evs]
-    full_ms, cached_ms = sum(full_each), sum(cached_each)
     assert qi.workspace_status(ws_f) == 0 and qi.workspace_status(ws_c) == 0
+    step_each = [e[0].elapsed_time(e[3]) for e in evs]
+    pos_each = [e[0].elapsed_time(e[1]) for e in evs]
+    full_each = [e[1].elapsed_time(e[2]) for e in evs]
+    cached_each = [e[2].elapsed_time(e[3]) for e in evs]
+    K = args.steps
+    step_ms = max_over_ranks(sum(step_each), world, dev)
+    full_ms = max_over_ranks(sum(full_each), world, dev)
+    cached_ms = max_over_ranks(sum(cached_each), world, dev)
+    peak = load_peaks()[0]["bf16_tflops"]
 
-    # ---- the projections of a cached step's target tokens (fused Q/K/V, output)
-    proj = time_projections(qi, args, B * T, H * 128, flush, dev)
+    def step_record(flops, ms_total, each):
+        tf = world * flops * K / (ms_total * 1e-3) / 1e12
+        return {"tflop": flops / 1e12, "ms": ms_total / K, "ms_median": pct(each, 50), "ms_p95": pct(each, 95),
+                "tflops": tf, "frac_of_peak": tf / peak / world}
 
-    # ---- the denoising loop (1 full + N-1 cached steps), eager and as a CUDA graph
-    loop = None
-    if cfg.get("cached_steps", 0) > 1 and not args.qk_norm:
-        loop = time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops)
+    rec = {"workload": W.DESCRIPTIONS[name], "B": B, "H": H, "L": L, "P": P, "T": T,
+           "full_step": step_record(full_flops, full_ms, full_each),
+           "cached_step": None if orig else step_record(cached_flops, cached_ms, cached_each),
+           "positions_ms_median": pct(pos_each, 50),
+           "step": {"ms": step_ms / K, "tflops": world * (full_flops + cached_flops) * K / (step_ms * 1e-3) / 1e12},
+           "gpu_launches": launches}
+    # per-rank throughput used for the line's aggregate value
+    raw = {"flops_per_step": full_flops + cached_flops, "step_ms": step_ms, "full_ms": full_ms,
+           "cached_ms": cached_ms, "launches": launches}
 
-    # ---- the whole denoising loop around the attention (optional: heavy)
-    dn = time_denoise(qi, args, cfg, dev) if args.denoise and not cfg.get("original") else None
+    if name == "maxref" and not args.qk_norm:
+        rec["loop"] = time_loop(qi, args, name, cfg, flush, dev, full_flops, cached_flops)
 
-    # ---- end to end through the C ABI with host buffers (copies timed)
-    h2d = sum(x.numel() * x.element_size() for x in host)
-    outs_d = [o_full] if orig else [o_full, o_c]
-    d2h = sum(o.numel() for o in outs_d) * 2
-    out_h = [torch.empty(o.shape, dtype=dt, pin_memory=True) for o in outs_d]
-    e2e_steps = max(3, min(args.steps, 20))
-    ee = [(mk(), mk()) for _ in range(e2e_steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(e2e_steps):
-        flush.zero_()
-        ee[i][0].record(stream)
-        for d, h in zip((dq, dk, dv, dqt, dkt, dvt), host):
-            d.copy_(h, non_blocking=True)
-        one_step()
-        for hh, dd in zip(out_h, outs_d):
-            hh.copy_(dd, non_blocking=True)
-        ee[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
+    if headline:
+        # end to end through the C ABI with host buffers: every step copies its
+        # inputs from pinned host memory and reads its outputs back (timed)
+        h2d = sum(x.numel() * x.element_size() for x in host)
+        outs_d = [o_full] if orig else [o_full, o_c]
+        d2h = sum(o.numel() for o in outs_d) * 2
+        out_h = [torch.empty(o.shape, dtype=dt, pin_memory=True) for o in outs_d]
+        e2e_steps = max(3, min(K, 20))
+        ee = [(mk(), mk()) for _ in range(e2e_steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in ee:
+            flush.zero_()
+            a.record(stream)
+            for d, h in zip((dq, dk, dv, dqt, dkt, dvt), host):
+                d.copy_(h, non_blocking=True)
+            one_step()
+            for hh, dd in zip(out_h, outs_d):
+                hh.copy_(dd, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), world, dev)
+        raw["e2e"] = {"value": world * (full_flops + cached_flops) * e2e_steps / (e2e_ms * 1e-3) / 1e12,
+                      "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "steps": e2e_steps}
+        if name == "t2i" or args.workload != "all":
+            rec["projections"] = time_projections(qi, args, B * T, H * 128, flush, dev)
+        if args.denoise and not orig:
+            rec["denoise"] = time_denoise(qi, args, cfg, dev)
+    elif name == "t2i":
+        rec["projections"] = time_projections(qi, args, B * T, H * 128, flush, dev)
+    del dq, dk, dv, dqt, dkt, dvt, kc, vc, o_full, o_c, ws_f, ws_c, host
+    torch.cuda.empty_cache()
+    return rec, raw
 
-    tot_flops = (full_flops + cached_flops) * args.steps
-    step_ms_max = max_over_ranks(step_ms, world, dev)
-    e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
-    all_flops = sum_over_ranks(tot_flops, world, dev)
-    all_e2e_flops = sum_over_ranks((full_flops + cached_flops) * e2e_steps, world, dev)
-    value = all_flops / (step_ms_max * 1e-3) / 1e12
-    e2e_value = all_e2e_flops / (e2e_ms_max * 1e-3) / 1e12
+
+def run_ours(args, world, rank, local):
+    import diffusion_transformer_joint_axial_b200 as qi
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    head = headline_workload(args)
+    names = BENCH_WORKLOADS if args.workload == "all" else (args.workload,)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    clocks = ClockSampler(dev) if rank == 0 else None
+    records, raw_head = {}, None
+    try:
+        for name in names:
+            assert W.WORKLOADS[name]["dtype"] == "bf16", "the bench measures the bf16 workloads"
+            rec, raw = bench_workload(qi, args, name, world, dev, flush, clocks, name == head)
+            records[name] = rec
+            if name == head:
+                raw_head = raw
+    finally:
+        clk = clocks.stop() if clocks else None
     if rank != 0:
         return
 
     peaks, kind = load_peaks()
-    # The burst peak fits kernels timed alone at full clock; a run that hit the
-    # power cap (long launches, e.g. the 2048^2 workload) is held to the
-    # sustained figure, measured the same way under the same cap.
-    capped = bool(clk) and "sw_power_cap" in clk.get("reasons", [])
-    if capped and "bf16_tflops_sustained" in peaks:
-        peak, peak_kind = peaks["bf16_tflops_sustained"], "%s bf16 dense sustained (cuBLAS under the power cap)" % kind
-    else:
-        peak, peak_kind = peaks["bf16_tflops"], "%s bf16 dense burst (cuBLAS)" % kind
-    att_ms = full_ms + cached_ms
-    achieved = (full_flops + cached_flops) * args.steps / (att_ms * 1e-3) / 1e12
-    full_tf = full_flops * args.steps / (full_ms * 1e-3) / 1e12
-    cached_tf = cached_flops * args.steps / (cached_ms * 1e-3) / 1e12 if cached_flops else None
+    peak = peaks["bf16_tflops"]
+    cfg = W.WORKLOADS[head]
+    L, P, T = W.sizes(head)
+    orig = cfg.get("original", False)
+    K = args.steps
+    hr = records[head]
+    value = hr["step"]["tflops"]
+    call_ms = raw_head["full_ms"] + raw_head["cached_ms"]
+    achieved = world * raw_head["flops_per_step"] * K / (call_ms * 1e-3) / 1e12 / world
 
     # the oracle baseline runs on rank 0 of a one-GPU run only
     budget = 0.0 if (args.no_cpu_baseline or world > 1) else args.cpu_budget
     cpu = None
     if budget > 0:
-        f, s, heads = oracle_sample(name, budget)
+        f, s, pieces = oracle_sample(head, budget)
         cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": "%d of %d (batch, head) pairs of the %s step (%s), float64 "
-                         "NumPy oracle, %.1f s" % (heads, B * H, name,
-                                                   "one unmasked full step" if orig else "full + one cached",
-                                                   s)}
+               "sample": "%d pieces of %d query rows of one head of the %s %s (float64 NumPy oracle, "
+                         "%.1f s; the rows cycle along the sequence)" % (
+                             pieces, ORACLE_ROWS, head,
+                             "unmasked full step" if orig else "full step + its cached step", s)}
+    power_note = None
+    if clk and "sw_power_cap" in (clk.get("reasons") or []):
+        power_note = ("sw_power_cap was active during the timed regions; the fractions still use the "
+                      "burst peak")
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms_max / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": hr["step"]["ms"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": W.DESCRIPTIONS[name], "B": B, "H": H, "L": L, "P": P, "T": T,
+        "config": {"workload": W.DESCRIPTIONS[head], "B": cfg["B"], "H": cfg["H"], "L": L, "P": P, "T": T,
                    "step": ("positions (text after the images) + one unmasked full step" if orig else
                             "positions + full block-causal step with cache store + one cached step")
                            + (", QK-RMSNorm fused (synthetic weights)" if args.qk_norm else ""),
+                   "timing": "whole C-ABI calls (rotation/cache pre-pass + attention kernel), CUDA events "
+                             "on the launch stream",
                    "qk_norm": bool(args.qk_norm),
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "dp%d (independent requests per GPU)" % world},
-        "full_step": {"tflops": full_tf, "frac_of_peak": full_tf / peak, "ms": full_ms / args.steps,
-                      "ms_median": pct(full_each, 50), "ms_p95": pct(full_each, 95)},
-        "cached_step": None if orig else {
-            "tflops": cached_tf, "frac_of_peak": cached_tf / peak, "ms": cached_ms / args.steps,
-            "ms_median": pct(cached_each, 50), "ms_p95": pct(cached_each, 95)},
+        "full_step": hr["full_step"],
+        "cached_step": hr["cached_step"],
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(name), "traffic_unit": "bytes/launch",
-                     "kernel": "qi21::tc::attn_tc_kernel (full + cached launches)",
-                     "peak_kind": peak_kind + ", MEASURED_PEAKS.json"},
+                     "frac": achieved / peak, "traffic": ncu_traffic(head), "traffic_unit": "bytes/call",
+                     "kernel": "attention calls of the step (full + cached): rotation/cache pre-pass + "
+                               "qi21::tc::attn_tc_kernel",
+                     "peak_kind": "%s bf16 dense burst (cuBLAS), MEASURED_PEAKS.json" % kind
+                                  if kind == "measured" else "fallback bf16 dense burst (1.59 PFLOP/s)"},
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": launches,
+        "e2e": raw_head["e2e"],
+        "gpu_launches": raw_head["launches"],
         "clocks": clk,
+        "power_note": power_note,
+        "workloads": records,
     }
-    line["projections"] = proj
-    if dn is not None:
-        line["denoise"] = dn
-    if loop is not None:
-        line["loop"] = loop
     print(json.dumps(line), flush=True)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="t2i", choices=[n for n in W.WORKLOADS if n != "tiny"])
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="all",
+                    choices=["all"] + [n for n in W.WORKLOADS if n != "tiny"],
+                    help="all (default): every bf16 workload, the 2048^2 one as the headline")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
