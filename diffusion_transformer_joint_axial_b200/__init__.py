@@ -10,11 +10,11 @@ from ._binding import (HEAD_DIM, LIB_PATH, QI21Error, Segment, alloc_cache, attn
                        cached_workspace_size, full_workspace_size, interleave_gate_up, launch_count, linear,
                        linear_residual, linear_swiglu,
                        load_library, new_workspace, rmsnorm, rope_positions, selftest_exp2,
-                       selftest_wait_timeout, swiglu, time_next_attention, workspace_status)
+                       selftest_wait_timeout, swiglu, workspace_status)
 from . import denoise
 from .steploop import DenoiseLoop
 
 __all__ = ["DenoiseLoop", "HEAD_DIM", "LIB_PATH", "QI21Error", "Segment", "alloc_cache", "attn_cached",
            "attn_full", "cached_workspace_size", "full_workspace_size", "interleave_gate_up", "launch_count",
            "linear", "linear_residual", "linear_swiglu", "load_library", "new_workspace", "rmsnorm", "rope_positions", "selftest_exp2",
-           "selftest_wait_timeout", "swiglu", "time_next_attention", "workspace_status"]
+           "selftest_wait_timeout", "swiglu", "workspace_status"]

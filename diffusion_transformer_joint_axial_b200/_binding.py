@@ -34,7 +34,7 @@ EXPORTED = (
     "qi21_linear", "qi21_linear_residual", "qi21_linear_swiglu", "qi21_rmsnorm", "qi21_swiglu",
     # status, errors, counters, timing and self-tests
     "qi21_workspace_status", "qi21_status_string", "qi21_last_error", "qi21_launch_count",
-    "qi21_time_next_attention", "qi21_selftest_wait_timeout", "qi21_selftest_exp2",
+    "qi21_selftest_wait_timeout", "qi21_selftest_exp2",
 )
 
 
@@ -98,8 +98,6 @@ def load_library(path=LIB_PATH):
     L.qi21_last_error.restype = ctypes.c_char_p
     L.qi21_launch_count.argtypes = []
     L.qi21_launch_count.restype = ctypes.c_uint64
-    L.qi21_time_next_attention.argtypes = [_vp, _vp]
-    L.qi21_time_next_attention.restype = None
     L.qi21_attn_cached_noalloc.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _vp, _vp]
     L.qi21_attn_cached_noalloc.restype = _i32
@@ -240,7 +238,7 @@ def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=
     if k_cache is not None:
         _need(k_cache, "k_cache", (B, H, P, HEAD_DIM), dt, dev)
         _need(v_cache, "v_cache", (B, H, P, HEAD_DIM), dt, dev)
-    need = full_workspace_size(B, H, L, P, dt)
+    need = full_workspace_size(B, H, L, P if k_cache is not None else 0, dt)
     if workspace is None:
         workspace = new_workspace(need, dev)
     norm = _norm_args(qk_norm, dev)
@@ -425,32 +423,32 @@ def swiglu(g, u, out=None):
     return out
 
 
-def workspace_status(workspace):
-    """Synchronises the current stream and returns (and clears) the status word."""
+def workspace_status(workspace, device=None):
+    """Synchronises the current stream and returns (and clears) the status word.
+
+    ``workspace=None`` reads the built-in scratch of the allocation-free
+    cached step (``qi21_attn_cached_noalloc``) on ``device`` (default: the
+    current one)."""
     L_ = _cuda_lib()
-    with torch.cuda.device(workspace.device):
-        return int(L_.qi21_workspace_status(_ptr(workspace), _stream(workspace.device)))
+    dev = workspace.device if workspace is not None else torch.device(
+        "cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    with torch.cuda.device(dev):
+        return int(L_.qi21_workspace_status(_ptr(workspace), _stream(dev)))
 
 
-def selftest_wait_timeout(workspace, limit_ns):
+def selftest_wait_timeout(workspace, limit_ns, device=None):
+    """One CTA waits (``limit_ns``) on a barrier nobody arrives at and records
+    the timeout in the workspace header (``None``: the built-in scratch)."""
     L_ = _cuda_lib()
-    with torch.cuda.device(workspace.device):
-        _check(L_.qi21_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(workspace.device)))
+    dev = workspace.device if workspace is not None else torch.device(
+        "cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(dev)))
 
 
 def launch_count():
     """Kernel launches this thread has enqueued through libqi21."""
     return int(load_library().qi21_launch_count())
-
-
-def time_next_attention(start, stop):
-    """Brackets the next attention-kernel launch with two torch CUDA events
-    (recorded on the kernel's own launch stream)."""
-    for e in (start, stop):
-        if e.cuda_event == 0:
-            e.record()  # torch creates the event lazily on first record
-    load_library().qi21_time_next_attention(ctypes.c_void_p(start.cuda_event),
-                                             ctypes.c_void_p(stop.cuda_event))
 
 
 def selftest_exp2(x):

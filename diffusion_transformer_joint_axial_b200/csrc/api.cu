@@ -12,7 +12,6 @@ namespace qi21 {
 
 static thread_local char g_last_error[512] = "";
 static thread_local uint64_t g_launches = 0;
-static thread_local cudaEvent_t g_time_start = nullptr, g_time_stop = nullptr;
 
 void note_launch() { ++g_launches; }
 
@@ -42,15 +41,17 @@ static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 static size_t elem_bytes(qi21_dtype dt) { return dt == QI21_F32 ? 4 : 2; }
 
-// Workspace: [header][cos/sin table: rows x 64 float2][rotated K: B x H x rows x 128]
+// Workspace: [header][cos/sin table: table_rows x 64 float2][rotated K: B x H x k_rows x 128]
+// (the query rows need the table; the key rows not stored in a cache need the
+// rotated-K room)
 struct WsLayout {
   size_t table_off, k_off, total;
 };
-static WsLayout ws_layout(int64_t B, int64_t H, int64_t rows, qi21_dtype dt) {
+static WsLayout ws_layout(int64_t B, int64_t H, int64_t table_rows, int64_t k_rows, qi21_dtype dt) {
   WsLayout w;
   w.table_off = QI21_WORKSPACE_HEADER_BYTES;
-  w.k_off = round_up(w.table_off + (size_t)rows * kPairs * sizeof(float2), 256);
-  w.total = round_up(w.k_off + (size_t)B * H * rows * kHeadDim * elem_bytes(dt), 256);
+  w.k_off = round_up(w.table_off + (size_t)table_rows * kPairs * sizeof(float2), 256);
+  w.total = round_up(w.k_off + (size_t)B * H * k_rows * kHeadDim * elem_bytes(dt), 256);
   return w;
 }
 
@@ -90,13 +91,8 @@ static qi21_status check_norm(const float* norm_q, const float* norm_k, float ep
 
 // Runs the attention kernel that matches the dtype.
 static qi21_status run_attention(const AttnArgs& a, qi21_dtype dt, cudaStream_t st) {
-  cudaEvent_t t0 = g_time_start, t1 = g_time_stop;
-  g_time_start = g_time_stop = nullptr;
-  cudaError_t e = cudaSuccess;
-  if (t0 != nullptr && t1 != nullptr) e = cudaEventRecord(t0, st);
-  if (e == cudaSuccess)
-    e = dt == QI21_F32 ? launch_attn_simt_f32(a, st) : launch_attn_tc_bf16(a, st, sm_count());
-  if (e == cudaSuccess && t0 != nullptr && t1 != nullptr) e = cudaEventRecord(t1, st);
+  const cudaError_t e =
+      dt == QI21_F32 ? launch_attn_simt_f32(a, st) : launch_attn_tc_bf16(a, st, sm_count());
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return QI21_OK;
 }
@@ -174,15 +170,14 @@ qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_seg
 }
 
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt) {
-  (void)P;
-  if (B < 0 || H < 0 || L < 0) return 0;
-  return ws_layout(B, H, L, dt).total;
+  if (B < 0 || H < 0 || L < 0 || P < 0 || P > L) return 0;
+  return ws_layout(B, H, L, L - P, dt).total;
 }
 
 size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt) {
   (void)P;
   if (B < 0 || H < 0 || T < 0) return 0;
-  return ws_layout(B, H, T, dt).total;
+  return ws_layout(B, H, T, T, dt).total;
 }
 
 static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
@@ -210,7 +205,9 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   QI21_TRY(check_norm(norm_q, norm_k, eps));
-  const WsLayout w = ws_layout(B, H, L, dt);
+  const bool cache = k_cache != nullptr && P > 0;
+  const int64_t split = cache ? P : L;
+  const WsLayout w = ws_layout(B, H, L, L - (cache ? P : 0), dt);
   if (workspace_bytes < w.total)
     return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -218,8 +215,6 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float2* table = reinterpret_cast<float2*>(ws + w.table_off);
   void* ws_k = ws + w.k_off;
-  const bool cache = k_cache != nullptr && P > 0;
-  const int64_t split = cache ? P : L;
 
   RopePrepParams rp;
   memset(&rp, 0, sizeof(rp));
@@ -290,7 +285,7 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(QI21_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   QI21_TRY(check_norm(norm_q, norm_k, eps));
-  const WsLayout w = ws_layout(B, H, T, dt);
+  const WsLayout w = ws_layout(B, H, T, T, dt);
   if (workspace_bytes < w.total)
     return fail(QI21_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -470,23 +465,31 @@ qi21_status qi21_swiglu(int64_t n, const void* g, const void* u, void* m, void* 
   return QI21_OK;
 }
 
+// NULL names the built-in scratch of qi21_attn_cached_noalloc.
+static qi21_status status_target(void** workspace) {
+  if (*workspace != nullptr) return QI21_OK;
+  const cudaError_t e = noalloc_scratch(workspace);
+  if (e != cudaSuccess) return cuda_fail(e, "built-in scratch address");
+  return QI21_OK;
+}
+
 qi21_status qi21_workspace_status(void* workspace, void* stream) {
-  if (workspace == nullptr) return fail(QI21_ERR_INVALID_ARG, "workspace is NULL");
+  QI21_TRY(status_target(&workspace));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WsHeader h;
   cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (h.status == QI21_OK) return QI21_OK;
-  const WsHeader zero = {0, 0};
-  e = cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
+  const uint32_t zero[2] = {0, 0};  // status and site; the schedule counter is left alone
+  e = cudaMemcpyAsync(workspace, zero, sizeof(zero), cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status clear");
   return fail(static_cast<qi21_status>(h.status), "device wait ran out (site 0x%x)", h.where);
 }
 
 qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream) {
-  QI21_TRY(check_ptr(workspace, "workspace"));
+  QI21_TRY(status_target(&workspace));
   if (limit_ns < 1 || limit_ns > 2000000000LL)
     return fail(QI21_ERR_INVALID_ARG, "limit_ns must be in [1, 2e9]");
   cudaError_t e = launch_wait_selftest(static_cast<uint32_t*>(workspace), (uint64_t)limit_ns,
@@ -502,11 +505,6 @@ qi21_status qi21_selftest_exp2(const float* x, float* y, int64_t n, void* stream
   cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "exp2 self-test launch");
   return QI21_OK;
-}
-
-void qi21_time_next_attention(void* start, void* stop) {
-  g_time_start = static_cast<cudaEvent_t>(start);
-  g_time_stop = static_cast<cudaEvent_t>(stop);
 }
 
 const char* qi21_status_string(qi21_status s) {

@@ -61,7 +61,7 @@ class DenoiseModel:
         # activations: every token (full path) and target tokens only (cached path)
         self.act = {n: self._acts(n) for n in ((L, T) if cached else (L,))}
         self.caches = [qb.alloc_cache(1, H, P, bf, dev) for _ in range(blocks)] if cached else None
-        self.ws_full = qb.new_workspace(qb.full_workspace_size(1, H, L, P, bf), dev)
+        self.ws_full = qb.new_workspace(qb.full_workspace_size(1, H, L, P if cached else 0, bf), dev)
         self.ws_cached = qb.new_workspace(qb.cached_workspace_size(1, H, P, T, bf), dev)
         self.ws_linear = qb.new_workspace(qb.WORKSPACE_HEADER_BYTES, dev)
         self.graph = None

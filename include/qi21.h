@@ -15,7 +15,11 @@
  *   contiguous [B, H, P, 128] (head-major).
  * - Pointers named "device" must be device memory of the current CUDA device;
  *   every device buffer must be 16-byte aligned.  The caller owns every buffer;
- *   the library allocates nothing and keeps no state between calls.
+ *   the library allocates nothing, and nothing one call leaves behind changes
+ *   what a later call computes: the only state it keeps is, per calling
+ *   thread, the last error message and a launch counter (the diagnostics at
+ *   the end of this header), plus the built-in scratch of
+ *   qi21_attn_cached_noalloc.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Calls validate their arguments on the host, enqueue kernels on `stream` and
  *   return without synchronising.  A failed launch returns QI21_ERR_CUDA.
@@ -24,6 +28,11 @@
  * - Device-side waits are bounded (about one second); a wait that runs out
  *   sets a status word in the workspace header and the kernel returns early.
  *   qi21_workspace_status() reads and clears that word.
+ * - Scratch: the attention calls take a caller-owned workspace (its header
+ *   holds the status word and the kernel's work counter; the rest holds the
+ *   per-token cos/sin table and the rotated keys of the call).  The paths
+ *   that need no workspace are qi21_rope_positions and
+ *   qi21_attn_cached_noalloc.
  */
 #ifndef QI21_H
 #define QI21_H
@@ -102,7 +111,10 @@ qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_
 qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_segs, int64_t L,
                                          int32_t* pos, int32_t* kv_end, void* stream);
 
-/* Workspace bytes qi21_attn_full needs for these sizes (header included). */
+/* Workspace bytes qi21_attn_full needs for these sizes (header included).
+ * P is the number of rows the call will store in a cache: pass the prefix
+ * length when k_cache/v_cache are given and 0 when they are not (the call
+ * checks workspace_bytes against the size for the rows it keeps). */
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt);
 
 /*
@@ -274,15 +286,16 @@ qi21_status qi21_swiglu(int64_t n, const void* g, const void* u, void* m, void* 
  * scratch is a 32 MiB array built into the library, held by every GPU that
  * loads the library until the process exits.  Calls needing more than that
  * (qi21_attn_cached_workspace_size() > 32 MiB) return QI21_ERR_INVALID_ARG
- * without enqueuing anything.  The first call on a device resolves the
- * array's device address (that device must be current); make that first call
- * before any stream capture.  No call allocates (no cudaMalloc/cudaFree).
- * Every call on a device shares the one array and the array keeps the last
- * call's contents: the call clears the status header itself, and calls whose
+ * without enqueuing anything; so does every other argument error.  Each call
+ * looks up the array's device address on the current device; the first call
+ * on a device also loads the library's device code there, so make it before
+ * any stream capture.  No call allocates (no cudaMalloc/cudaFree).  Every
+ * call on a device shares the one array and the array keeps the last call's
+ * contents (a call resets what must start at zero itself), so calls whose
  * kernels overlap on the GPU (other streams, other threads) race on the
  * scratch -- order them on one stream.  A device wait that runs out is
- * recorded in that header but cannot be read back; callers needing that
- * report use qi21_attn_cached with a workspace.
+ * recorded in the array's status header and stays there until
+ * qi21_workspace_status(NULL, stream) reads and clears it.
  */
 qi21_status qi21_attn_cached_noalloc(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
                                      const void* q, const void* k, const void* v,
@@ -290,13 +303,21 @@ qi21_status qi21_attn_cached_noalloc(int32_t B, int32_t H, int64_t P, int64_t T,
                                      const void* v_cache, void* o, void* stream);
 
 /* Synchronises `stream`, then reads and clears the status word in the
- * workspace header: QI21_OK, or QI21_ERR_TIMEOUT if a device wait ran out. */
+ * workspace header: QI21_OK, or QI21_ERR_TIMEOUT if a device wait ran out.
+ * workspace = NULL reads the built-in scratch of qi21_attn_cached_noalloc on
+ * the current device. */
 qi21_status qi21_workspace_status(void* workspace, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics and test support.  Not part of the computation: a test hook for
+ * the bounded waits, the message of the last error and a launch counter.
+ * ------------------------------------------------------------------------- */
 
 /* Test hook for the bounded-wait machinery: launches one CTA that waits on a
  * shared-memory barrier nobody arrives at, with a limit of `limit_ns`
  * nanoseconds (1..2e9).  The kernel records QI21_ERR_TIMEOUT in the workspace
- * header and exits normally; read it with qi21_workspace_status(). */
+ * header (workspace = NULL: the built-in scratch of qi21_attn_cached_noalloc)
+ * and exits normally; read it with qi21_workspace_status(). */
 qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
 
 /* Test hook for the polynomial exp2 that the bf16 softmax evaluates on the
@@ -304,14 +325,6 @@ qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* 
  * cubic minimax fit, relative error below 1e-4 for x in [-125, 128)).
  * Writes y[i] = 2^x[i] for n device floats (x clamped below at -125). */
 qi21_status qi21_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
-
-/* Profiling hook.  When `start` and `stop` are cudaEvent_t handles (passed
- * as void*), the next attention-kernel launch made by this thread (through
- * qi21_attn_full or qi21_attn_cached) is bracketed by cudaEventRecord(start)
- * and cudaEventRecord(stop) on its launch stream -- the attention kernel only,
- * not the rotation pre-pass -- after which the hook clears itself.  NULLs turn
- * it off.  The events stay owned by the caller. */
-void qi21_time_next_attention(void* start, void* stop);
 
 const char* qi21_status_string(qi21_status s);
 

@@ -41,7 +41,7 @@ def gpu_full(segments, q, k, v, P, cache=True, device="cuda"):
     kc = vc = None
     if cache:
         kc, vc = qi.alloc_cache(B, H, P, q.dtype, dev)
-    ws = qi.new_workspace(qi.full_workspace_size(B, H, L, P, q.dtype), dev)
+    ws = qi.new_workspace(qi.full_workspace_size(B, H, L, P if cache else 0, q.dtype), dev)
     o = qi.attn_full(qd, kd, vd, pos, kv_end, P, kc, vc, workspace=ws)
     check_status(ws)
     torch.cuda.synchronize()

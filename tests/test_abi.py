@@ -49,9 +49,14 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     full = lib.qi21_attn_full_workspace_size(1, 24, 4352, 256, qb.QI21_BF16)
-    # header + cos/sin table (L x 64 float2) + rotated keys (B x H x L x 128 bf16)
-    assert full >= 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
+    # header + cos/sin table (L x 64 float2) + rotated keys of the rows not
+    # stored in the cache (B x H x (L - P) x 128 bf16)
+    assert full >= 256 + 4352 * 64 * 8 + 24 * 4096 * 128 * 2
+    assert full < 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
     assert full % 256 == 0
+    no_cache = lib.qi21_attn_full_workspace_size(1, 24, 4352, 0, qb.QI21_BF16)
+    assert no_cache >= 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
+    assert lib.qi21_attn_full_workspace_size(1, 24, 4352, 4353, qb.QI21_BF16) == 0  # P > L
     cached = lib.qi21_attn_cached_workspace_size(1, 24, 256, 4096, qb.QI21_BF16)
     assert cached >= 256 + 4096 * 64 * 8 + 24 * 4096 * 128 * 2
     assert lib.qi21_attn_full_workspace_size(-1, 1, 1, 0, 0) == 0
