@@ -34,7 +34,7 @@ EXPORTED = (
     "qi21_linear", "qi21_linear_residual", "qi21_linear_swiglu", "qi21_rmsnorm", "qi21_swiglu",
     # status, errors, counters, timing and self-tests
     "qi21_workspace_status", "qi21_status_string", "qi21_last_error", "qi21_launch_count",
-    "qi21_selftest_wait_timeout", "qi21_selftest_exp2",
+    "qi21_selftest_wait_timeout",
 )
 
 
@@ -101,8 +101,6 @@ def load_library(path=LIB_PATH):
     L.qi21_attn_cached_noalloc.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _vp, _vp]
     L.qi21_attn_cached_noalloc.restype = _i32
-    L.qi21_selftest_exp2.argtypes = [_vp, _vp, _i64, _vp]
-    L.qi21_selftest_exp2.restype = _i32
     for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached", "qi21_attn_full_qknorm",
                  "qi21_attn_cached_qknorm", "qi21_workspace_status", "qi21_selftest_wait_timeout"):
         getattr(L, name).restype = _i32
@@ -449,13 +447,3 @@ def selftest_wait_timeout(workspace, limit_ns, device=None):
 def launch_count():
     """Kernel launches this thread has enqueued through libqi21."""
     return int(load_library().qi21_launch_count())
-
-
-def selftest_exp2(x):
-    """The softmax's polynomial exp2 evaluated on a float32 CUDA tensor."""
-    L_ = _cuda_lib()
-    x = x.contiguous()
-    y = torch.empty_like(x)
-    with torch.cuda.device(x.device):
-        _check(L_.qi21_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(x.device)))
-    return y

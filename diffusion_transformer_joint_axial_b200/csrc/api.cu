@@ -498,15 +498,6 @@ qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* 
   return QI21_OK;
 }
 
-qi21_status qi21_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
-  if (n < 0) return fail(QI21_ERR_INVALID_ARG, "n must be >= 0");
-  if (n == 0) return QI21_OK;
-  if (x == nullptr || y == nullptr) return fail(QI21_ERR_INVALID_ARG, "x and y must not be NULL");
-  cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "exp2 self-test launch");
-  return QI21_OK;
-}
-
 const char* qi21_status_string(qi21_status s) {
   switch (s) {
     case QI21_OK: return "QI21_OK";

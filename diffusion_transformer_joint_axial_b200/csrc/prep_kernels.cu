@@ -327,27 +327,4 @@ cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream
   return cudaGetLastError();
 }
 
-// ============================================================ exp2 test ==
-// Evaluates the polynomial exp2 the attention softmax uses on part of its
-// columns, so tests can compare it with exp2 in float64 and with CUDA's own.
-__global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
-  const int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
-    y[i] = r.x;
-    y[i + 1] = r.y;
-  } else if (i < n) {
-    y[i] = exp2_poly2(make_float2(x[i], x[i])).x;
-  }
-}
-
-cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t stream) {
-  if (n == 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t blocks = ((n + 1) / 2 + threads - 1) / threads;
-  exp2_poly_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, y, n);
-  note_launch();
-  return cudaGetLastError();
-}
-
 }  // namespace qi21

@@ -103,6 +103,9 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint3
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -223,28 +226,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(v);
-}
-
-// 2^x for a pair, on the FMA/ALU pipes.  Range reduction x = j + f with
-// j = round(x) (the 1.5 * 2^23 rounding constant leaves j in the low bits of
-// t), f in [-1/2, 1/2]; 2^f from a cubic minimax fit (Remez exchange on the
-// relative error, max 7.5e-5 = 2^-13.7, far below bf16's 2^-9); 2^j is added
-// straight into the exponent field.  x is clamped to >= -125 so the result
-// stays a normal float; callers use it only where x is finite.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-  float2 p = __ffma2_rn(f, make_float2(0.0551716685295105f, 0.0551716685295105f),
-                        make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  const uint32_t rx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-  const uint32_t ry = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 }  // namespace qi21

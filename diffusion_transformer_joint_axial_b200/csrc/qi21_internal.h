@@ -122,7 +122,6 @@ cudaError_t launch_swiglu(int64_t n, const void* g, const void* u, void* m, cuda
 
 // --------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
-cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 // Device address of qi21_attn_cached_noalloc's built-in scratch on the
 // current device (noalloc.cu).

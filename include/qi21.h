@@ -320,12 +320,6 @@ qi21_status qi21_workspace_status(void* workspace, void* stream);
  * and exits normally; read it with qi21_workspace_status(). */
 qi21_status qi21_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
 
-/* Test hook for the polynomial exp2 that the bf16 softmax evaluates on the
- * FMA pipe for part of its columns (range reduction to [-1/2, 1/2] plus a
- * cubic minimax fit, relative error below 1e-4 for x in [-125, 128)).
- * Writes y[i] = 2^x[i] for n device floats (x clamped below at -125). */
-qi21_status qi21_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
-
 const char* qi21_status_string(qi21_status s);
 
 /* Message describing the last non-OK status returned to the calling thread. */
