@@ -90,6 +90,7 @@ constexpr float kRescaleRaw = 8.0f / kScaleLog2;
 
 struct Params {
   CUtensorMap tm_q;
+  CUtensorMap tm_o;  // the output: 64 columns x 32 rows boxes (one epilogue warp's rows)
   CUtensorMap tm_k0, tm_k1, tm_v0, tm_v1;
   int32_t k0_tok, k1_tok, v0_tok, v1_tok;  // 1: token-major coords, 0: head-major
   int32_t B, H, Lq, n0, n1;
@@ -112,6 +113,9 @@ struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
+  // 64 columns x 128 rows of O (bf16, 128B-swizzled): each epilogue warp
+  // stages its 32 rows (4 KB) here for its own TMA store
+  uint8_t ostage[kHalfBytes];
   float row_l[2][2][BM];  // [unit parity][tile][row]: softmax -> epilogue
   alignas(16) float qnw[kHeadDim];  // QK-RMSNorm weight of Q (when given)
   int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
@@ -443,6 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (p.q_norm_w != nullptr && threadIdx.x < kHeadDim) S.qnw[threadIdx.x] = p.q_norm_w[threadIdx.x];
   if (warp == kWarpLoad && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_o);
     tma_prefetch_desc(&p.tm_k0);
     tma_prefetch_desc(&p.tm_v0);
     if (p.n1 > 0) {
@@ -704,19 +709,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                               p.status, 0x410 | s));
         if (!ok) break;
         tc_fence_after();
-        const int row = prev.row0 + s * BM + t;
-        const bool valid = row < p.Lq;
         const float inv = 1.f / S.row_l[par][s][t];
-        __nv_bfloat16* dst =
-            p.o + (((size_t)prev.b * p.Lq + (valid ? row : 0)) * p.H + prev.h) * kHeadDim;
         const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
+        // O / l -> bf16 in two 64-column halves.  Each warp stages its own 32
+        // rows in shared memory (128B-swizzled, the TMA layout) and writes
+        // them with one TMA store (rows past Lq are clipped; a box wholly past
+        // Lq is not issued).  O's TMEM columns are released as soon as the
+        // second half has been read, long before the stores finish.  No
+        // barrier spans warps, so a warp that gives up on a timed-out wait
+        // cannot hold the others.
+        uint8_t* stage = S.ostage + (warp & 3) * 32 * 128;
+        const int row_first = prev.row0 + s * BM + (warp & 3) * 32;
+        for (int hh = 0; hh < 2; ++hh) {
+          if (lane == 0) bulk_wait_read_all();  // this warp's slice of the stage is free
+          __syncwarp();
 #pragma unroll 1
-        for (int c = 0; c < kHeadDim; c += 32) {
-          uint32_t orow[32];
-          tmem_ld32(tO + c, orow);
-          tmem_wait_ld();
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(tO + 64 * hh + 32 * c, orow);
+            tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               uint32_t w[4];
@@ -724,17 +735,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               for (int i = 0; i < 4; ++i)
                 w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
                                    __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
-              d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+              const int chunk = 4 * c + e;  // 16-byte chunk of the 128-byte row
+              *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&S.o_free[s]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row_first < p.Lq) {
+            tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, prev.h, row_first, prev.b);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&S.o_free[s]));
       }
       if (u < 0) break;
       prev = U;
       have_prev = true;
     }
+    // the shared-memory stage must stay valid until the last stores read it
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
     setmaxnreg_inc_softmax();
@@ -883,7 +908,8 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   tc::Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t tok = (uint64_t)a.H * kHeadDim * 2;
-  if (!encode_4d(&p.tm_q, a.q, a.H, a.Lq, a.B, kHeadDim * 2, tok, tok * a.Lq, 1, tc::BM))
+  if (!encode_4d(&p.tm_q, a.q, a.H, a.Lq, a.B, kHeadDim * 2, tok, tok * a.Lq, 1, tc::BM) ||
+      !encode_4d(&p.tm_o, a.o, a.H, a.Lq, a.B, kHeadDim * 2, tok, tok * a.Lq, 1, 32))
     return cudaErrorInvalidValue;
   if (!encode_source(&p.tm_k0, a.k0, a.B, a.H, &p.k0_tok) ||
       !encode_source(&p.tm_k1, a.k1, a.B, a.H, &p.k1_tok) ||
