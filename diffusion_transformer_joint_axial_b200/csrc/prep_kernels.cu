@@ -66,9 +66,6 @@ cudaError_t launch_positions(const PositionsParams& p, cudaStream_t stream) {
 // With a K norm weight, each head row is first divided by its root mean
 // square (plus eps under the root) and multiplied by the weight: the
 // QK-RMSNorm that precedes RoPE (overview card 4A; close reading section 6).
-// Work split: a CTA takes four tokens of one batch; its K chunks are numbered
-// (token, head, chunk) and dealt to the threads round-robin, the first loads
-// going out before the float64 angles are computed.
 
 Omega make_omega() {
   Omega o;
@@ -81,7 +78,6 @@ Omega make_omega() {
 
 constexpr int kPrepTokens = 4;  // tokens per CTA
 constexpr int kPrepThreads = 256;
-constexpr int kPrepUnroll = 4;  // 16-byte loads each thread keeps in flight
 
 template <typename T>
 struct Vec16;  // 16-byte vector of T
@@ -151,138 +147,120 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
-// One 16-byte chunk of the work: token t of the CTA, head h, chunk c of the
-// head row.  The chunks of one row are CPR consecutive work items, so they
-// sit in CPR consecutive lanes.
-struct PrepItem {
-  int t, h, c;
-};
-template <int CPR>
-__device__ __forceinline__ PrepItem prep_item(int e, int H, float inv_h) {
-  PrepItem it;
-  const int r = e / CPR;  // row (t, h); CPR is a power of two
-  it.c = e - r * CPR;
-  // r / H through the reciprocal: exact for the few rows of one CTA
-  it.t = static_cast<int>((static_cast<float>(r) + 0.5f) * inv_h);
-  it.h = r - it.t * H;
-  return it;
-}
+// Thread layout: a CTA takes kPrepTokens tokens of one batch.  Thread i keeps
+// one 16-byte chunk c = i % CPR of the head rows of one token and walks that
+// token's heads h0, h0 + SPT, h0 + 2 SPT, ... (SPT head slots per token), so
+// the chunk's (cos, sin) pairs are read once and reused for every head, and
+// consecutive lanes cover consecutive bytes of a row (coalesced).
+constexpr int kPrepHeadsInFlight = 8;  // head rows whose loads a thread keeps in flight
 
 template <typename T>
 __global__ void __launch_bounds__(kPrepThreads)
     rope_prep_kernel(const __grid_constant__ RopePrepParams p) {
-  __shared__ float2 cs[kPrepTokens][kPairs];
+  __shared__ __align__(16) float2 cs[kPrepTokens][kPairs];
   __shared__ __align__(16) float wn[kHeadDim];  // norm weight of K
-  constexpr int EPC = Vec16<T>::N;     // elements per 16-byte chunk
-  constexpr int CPR = kHeadDim / EPC;  // chunks per head row
+  constexpr int EPC = Vec16<T>::N;       // elements per 16-byte chunk
+  constexpr int CPR = kHeadDim / EPC;    // chunks per head row (a power of two)
+  constexpr int SLOTS = kPrepThreads / CPR;
+  constexpr int SPT = SLOTS / kPrepTokens;  // head slots per token
+  static_assert(SPT >= 1 && SLOTS % kPrepTokens == 0, "thread layout");
   const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kPrepTokens;
   const int b = blockIdx.y;
-  const int lane = threadIdx.x & 31;
+  const int c = threadIdx.x % CPR;
+  const int slot = threadIdx.x / CPR;
+  const int t = slot / SPT;
+  const int h0 = slot % SPT;
+  const int64_t tok = tok0 + t;
+  const int H = p.H;
+  const bool has_tok = tok < p.Lk;
+  const int iters = (H + SPT - 1) / SPT;  // the same for every thread (shuffle reductions)
   if (p.unit_counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
     *p.unit_counter = 0u;
-  const int ntok = static_cast<int>(p.Lk - tok0 < kPrepTokens ? p.Lk - tok0 : kPrepTokens);
-  const int H = p.H;
-  const int items = ntok * H * CPR;
-  const float inv_h = 1.0f / static_cast<float>(H);
   const bool norm = p.k_norm_w != nullptr;
-  const T* __restrict__ k = static_cast<const T*>(p.k);
+  const T* __restrict__ kp = static_cast<const T*>(p.k) + ((static_cast<int64_t>(b) * p.Lk + tok) * H) *
+                                                              kHeadDim + c * EPC;
+  // destination of this token's rows: the cache for the first `split` tokens, the rest after
+  const bool first = tok < p.split;
+  T* const dst_base = static_cast<T*>(first ? p.k_dst0 : p.k_dst1);
+  const int64_t rows = first ? p.split : p.Lk - p.split;
+  const int64_t row = first ? tok : tok - p.split;
 
   // The first loads go out before the angles are computed: they do not need them.
-  uint4 x[kPrepUnroll];
-  auto issue = [&](int e0) {
+  uint4 x[kPrepHeadsInFlight];
+  auto load_batch = [&](int i0) {
 #pragma unroll
-    for (int i = 0; i < kPrepUnroll; ++i) {
-      const int e = e0 + i * kPrepThreads;
-      if (e < items) {
-        const PrepItem it = prep_item<CPR>(e, H, inv_h);
-        x[i] = ld_stream(k + ((static_cast<int64_t>(b) * p.Lk + tok0 + it.t) * H + it.h) * kHeadDim +
-                         it.c * EPC);
-      }
+    for (int j = 0; j < kPrepHeadsInFlight; ++j) {
+      const int h = h0 + (i0 + j) * SPT;
+      if (has_tok && i0 + j < iters && h < H) x[j] = ld_stream(kp + static_cast<int64_t>(h) * kHeadDim);
     }
   };
-  issue(threadIdx.x);
+  load_batch(0);
 
   if (norm && threadIdx.x < kHeadDim) wn[threadIdx.x] = p.k_norm_w[threadIdx.x];
   if (threadIdx.x < kPrepTokens * kPairs) {
-    const int t = threadIdx.x / kPairs, m = threadIdx.x % kPairs;
-    if (t < ntok) {
+    const int tt = threadIdx.x / kPairs, m = threadIdx.x % kPairs;
+    if (tok0 + tt < p.Lk) {
       const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
-      const double ang = static_cast<double>(p.pos[3 * (tok0 + t) + axis]) * p.omega.w[m];
+      const double ang = static_cast<double>(p.pos[3 * (tok0 + tt) + axis]) * p.omega.w[m];
       double sd, cd;
       sincos(ang, &sd, &cd);
       const float2 v = make_float2(static_cast<float>(cd), static_cast<float>(sd));
-      cs[t][m] = v;
+      cs[tt][m] = v;
       if (p.table != nullptr && b == 0) {
         if (p.table_half)
-          static_cast<__half2*>(p.table)[(tok0 + t) * kPairs + m] = __halves2half2(__double2half(cd), __double2half(sd));
+          static_cast<__half2*>(p.table)[(tok0 + tt) * kPairs + m] = __halves2half2(__double2half(cd), __double2half(sd));
         else
-          static_cast<float2*>(p.table)[(tok0 + t) * kPairs + m] = v;
+          static_cast<float2*>(p.table)[(tok0 + tt) * kPairs + m] = v;
       }
     }
   }
   __syncthreads();
-
-  // The loop runs while any lane of the warp has work, so that every lane
-  // takes part in the norm's shuffle reduction (a row's CPR chunks are CPR
-  // consecutive lanes: CPR divides 32 and the thread count).
-  for (int e0 = threadIdx.x; e0 - lane < items; e0 += kPrepUnroll * kPrepThreads) {
-    if (e0 != static_cast<int>(threadIdx.x)) issue(e0);
+  // this chunk's (cos, sin) pairs, the same for every head of the token
+  float2 r[EPC / 2];
 #pragma unroll
-    for (int i = 0; i < kPrepUnroll; ++i) {
-      const int e = e0 + i * kPrepThreads;
+  for (int e = 0; e < EPC / 2; ++e) r[e] = cs[t][c * (EPC / 2) + e];
+  const float* wc = norm ? &wn[c * EPC] : nullptr;
+
+  for (int i0 = 0; i0 < iters; i0 += kPrepHeadsInFlight) {
+    if (i0 > 0) load_batch(i0);
+#pragma unroll
+    for (int j = 0; j < kPrepHeadsInFlight; ++j) {
+      if (i0 + j >= iters) break;
+      const int h = h0 + (i0 + j) * SPT;
+      const bool live = has_tok && h < H;
       float rs = 1.f;
       if (norm) {
-        float ss = e < items ? sumsq_chunk(x[i], static_cast<T*>(nullptr)) : 0.f;
+        // the row's CPR chunks are CPR consecutive lanes
+        float ss = live ? sumsq_chunk(x[j], static_cast<T*>(nullptr)) : 0.f;
 #pragma unroll
         for (int o = CPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         rs = rsqrtf(ss * (1.f / kHeadDim) + p.norm_eps);
       }
-      if (e >= items) continue;
-      const PrepItem it = prep_item<CPR>(e, H, inv_h);
-      const int64_t tok = tok0 + it.t;
-      rotate_chunk(x[i], &cs[it.t][it.c * EPC / 2], rs, norm ? &wn[it.c * EPC] : nullptr,
-                   static_cast<T*>(nullptr));
-      T* dst;
-      int64_t row, rows;
-      if (tok < p.split) {
-        dst = static_cast<T*>(p.k_dst0);
-        row = tok;
-        rows = p.split;
-      } else {
-        dst = static_cast<T*>(p.k_dst1);
-        row = tok - p.split;
-        rows = p.Lk - p.split;
-      }
-      *reinterpret_cast<uint4*>(dst + ((static_cast<int64_t>(b) * H + it.h) * rows + row) * kHeadDim +
-                                it.c * EPC) = x[i];
+      if (!live) continue;
+      rotate_chunk(x[j], r, rs, wc, static_cast<T*>(nullptr));
+      *reinterpret_cast<uint4*>(dst_base + ((static_cast<int64_t>(b) * H + h) * rows + row) * kHeadDim +
+                                c * EPC) = x[j];
     }
   }
 
   // Prefix V rows: a plain copy into the V cache.
-  if (p.v_dst0 != nullptr && tok0 < p.split) {
-    const int nv = static_cast<int>(p.split - tok0 < ntok ? p.split - tok0 : ntok);
-    const int vitems = nv * H * CPR;
-    const T* __restrict__ v = static_cast<const T*>(p.v);
-    for (int e0 = threadIdx.x; e0 < vitems; e0 += kPrepUnroll * kPrepThreads) {
-      uint4 y[kPrepUnroll];
+  if (p.v_dst0 != nullptr && has_tok && first) {
+    const T* __restrict__ vp = static_cast<const T*>(p.v) + ((static_cast<int64_t>(b) * p.Lk + tok) * H) *
+                                                                kHeadDim + c * EPC;
+    T* const vd = static_cast<T*>(p.v_dst0);
+    for (int i0 = 0; i0 < iters; i0 += kPrepHeadsInFlight) {
+      uint4 y[kPrepHeadsInFlight];
 #pragma unroll
-      for (int i = 0; i < kPrepUnroll; ++i) {
-        const int e = e0 + i * kPrepThreads;
-        if (e < vitems) {
-          const PrepItem it = prep_item<CPR>(e, H, inv_h);
-          y[i] = ld_stream(v + ((static_cast<int64_t>(b) * p.Lk + tok0 + it.t) * H + it.h) * kHeadDim +
-                           it.c * EPC);
-        }
+      for (int j = 0; j < kPrepHeadsInFlight; ++j) {
+        const int h = h0 + (i0 + j) * SPT;
+        if (i0 + j < iters && h < H) y[j] = ld_stream(vp + static_cast<int64_t>(h) * kHeadDim);
       }
 #pragma unroll
-      for (int i = 0; i < kPrepUnroll; ++i) {
-        const int e = e0 + i * kPrepThreads;
-        if (e < vitems) {
-          const PrepItem it = prep_item<CPR>(e, H, inv_h);
-          *reinterpret_cast<uint4*>(static_cast<T*>(p.v_dst0) +
-                                    ((static_cast<int64_t>(b) * H + it.h) * p.split + tok0 + it.t) * kHeadDim +
-                                    it.c * EPC) = y[i];
-        }
+      for (int j = 0; j < kPrepHeadsInFlight; ++j) {
+        const int h = h0 + (i0 + j) * SPT;
+        if (i0 + j < iters && h < H)
+          *reinterpret_cast<uint4*>(vd + ((static_cast<int64_t>(b) * H + h) * p.split + tok) * kHeadDim +
+                                    c * EPC) = y[j];
       }
     }
   }
