@@ -39,10 +39,8 @@
 // eight-chain row max): on B200 a lone softmax warp per SMSP is bound by
 // instruction latency more than by the MUFU exp2 rate.
 // Online softmax uses a lazy rescale: O and l are rescaled only when a row
-// maximum grows by more than 2^8, which keeps every P <= 256.  Past the first
-// key tile the exponentials of a tile's first half start from the running
-// maximum while the tile's own maximum is computed beside them; the rare row
-// whose maximum grows past the threshold redoes that half.
+// maximum grows by more than 2^8, which keeps every P <= 256.  Each tile's
+// row maximum is taken before its exponentials.
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <math.h>
