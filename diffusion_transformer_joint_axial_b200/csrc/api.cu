@@ -55,6 +55,27 @@ static WsLayout ws_layout(int64_t B, int64_t H, int64_t table_rows, int64_t k_ro
   return w;
 }
 
+// Tail-split scratch of a cached step (the attention's last, partial wave of
+// units split into key-range pieces): arrival counters for up to
+// kSplitUnitsCap units, then per piece slot 64 KB of O / l (bf16) and 2 KB of
+// (row max, row sum).  Slots: up to four per unit, at most kSplitSlotsCap.
+constexpr int64_t kSplitUnitsCap = 512;
+constexpr int64_t kSplitSlotsCap = 512;
+constexpr size_t kSplitSlotPartBytes = (size_t)2 * 128 * kHeadDim * 2;
+constexpr size_t kSplitSlotMlBytes = (size_t)2 * 128 * sizeof(float2);
+struct SplitCaps {
+  int64_t units, slots;
+  size_t cnt_bytes;
+};
+static SplitCaps split_caps(int64_t B, int64_t H, int64_t T) {
+  const int64_t units = B * H * ((T + 255) / 256);
+  SplitCaps c;
+  c.units = units < kSplitUnitsCap ? units : kSplitUnitsCap;
+  c.slots = 4 * units < kSplitSlotsCap ? 4 * units : kSplitSlotsCap;
+  c.cnt_bytes = round_up((size_t)c.units * 8 * sizeof(uint32_t), 256);
+  return c;
+}
+
 static int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -95,6 +116,11 @@ static qi21_status run_attention(const AttnArgs& a, qi21_dtype dt, cudaStream_t 
       dt == QI21_F32 ? launch_attn_simt_f32(a, st) : launch_attn_tc_bf16(a, st, sm_count());
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return QI21_OK;
+}
+
+size_t attn_cached_workspace_min(int32_t B, int32_t H, int64_t T, qi21_dtype dt) {
+  if (B < 0 || H < 0 || T < 0) return 0;
+  return ws_layout(B, H, T, T, dt).total;
 }
 
 }  // namespace qi21
@@ -177,7 +203,10 @@ size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P,
 size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt) {
   (void)P;
   if (B < 0 || H < 0 || T < 0) return 0;
-  return ws_layout(B, H, T, T, dt).total;
+  const size_t base = ws_layout(B, H, T, T, dt).total;
+  if (dt != QI21_BF16 || B == 0 || H == 0 || T == 0) return base;
+  const SplitCaps c = split_caps(B, H, T);
+  return base + c.cnt_bytes + (size_t)c.slots * (kSplitSlotPartBytes + kSplitSlotMlBytes);
 }
 
 static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
@@ -310,12 +339,30 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;
   rp.norm_eps = eps;
+
+  // Tail-split scratch: whatever the workspace holds past the minimum layout
+  // (none: the call runs unsplit).
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  if (dt == QI21_BF16) {
+    const SplitCaps c = split_caps(B, H, T);
+    const size_t avail = workspace_bytes - w.total;
+    if (avail >= c.cnt_bytes + kSplitSlotPartBytes + kSplitSlotMlBytes) {
+      int64_t slots = (int64_t)((avail - c.cnt_bytes) / (kSplitSlotPartBytes + kSplitSlotMlBytes));
+      if (slots > c.slots) slots = c.slots;
+      a.split_cnt = reinterpret_cast<uint32_t*>(ws + w.total);
+      a.split_cnt_units = (int32_t)c.units;
+      a.split_part = ws + w.total + c.cnt_bytes;
+      a.split_ml = ws + w.total + c.cnt_bytes + (size_t)slots * kSplitSlotPartBytes;
+      a.split_slots = (int32_t)slots;
+      rp.zero_words = a.split_cnt;
+      rp.n_zero_words = (int32_t)(c.units * 8);
+    }
+  }
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
   const int64_t tokstride = (int64_t)H * kHeadDim;
-  AttnArgs a;
-  memset(&a, 0, sizeof(a));
   a.unit_counter = rp.unit_counter;
   a.B = B;
   a.H = H;

@@ -11,6 +11,12 @@
 // per SM, persistent) take units from a global counter in order of decreasing
 // cost (longest-processing-time-first, decided at run time), heads grouped so
 // that concurrent CTAs share K/V in L2.
+// Without a mask (the cached step) every unit costs the same, and the units of
+// the last, partial wave can leave most SMs idle (384 units on 148 SMs are 2.6
+// waves); there the host may hand those units out as k key-range pieces each
+// (chosen by a cost model): each piece writes its O / l (bf16) and its row
+// max and row sum to the workspace, and the epilogue warp that finishes the
+// last piece of a unit's rows (an arrival counter, no waiting) merges them.
 // For each query tile only the key tiles that start below the tile's largest
 // kv_end are visited: every visibility bound is a prefix of the keys, so
 // fully masked tiles are skipped and never loaded; only tiles that straddle
@@ -18,16 +24,18 @@
 // element-wise.
 //
 // Warp roles (512 threads, registers rebalanced with setmaxnreg):
-//   warps 0-3   softmax for query tile 0 (thread = row = TMEM lane), 168 regs
-//   warps 4-7   softmax for query tile 1, 168 regs
-//   warps 8-11  Q rotation and epilogue (O / l -> bf16 -> global) for both
-//               tiles, 72 regs: each unit's query tiles are rotated as soon
-//               as they land, before the previous unit's O is drained, so
-//               the rotation overlaps the previous unit's last key tiles
-//   warp  12    TMA producer of Q tiles and the K ring (2 stages), 104 regs
-//   warp  13    TMEM allocator and tcgen05.mma issuer, 104 regs
-//   warp  14    TMA producer of the V ring (2 stages), 104 regs
-//   warp  15    idle, 104 regs
+//   warps 0-3   query tile 0: rotates each item's query rows in shared memory
+//               once the tile lands (one row per thread, its cos/sin chunks
+//               requested before the wait), then the softmax (thread = row =
+//               TMEM lane), 160 regs
+//   warps 4-7   the same for query tile 1, 160 regs
+//   warps 8-11  epilogue, 80 regs: drains each item's O (O / l -> bf16 ->
+//               TMA store, or a piece's partial result and the merge) as soon
+//               as its MMAs are done
+//   warp  12    TMA producer of Q tiles and the K ring (2 stages), 112 regs
+//   warp  13    TMEM allocator and tcgen05.mma issuer, 112 regs
+//   warp  14    TMA producer of the V ring (2 stages), 112 regs
+//   warp  15    idle, 112 regs
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the upper 64 columns of its S and is the A
 // operand of the P*V MMA, so P never touches shared memory.  P is released in
@@ -63,10 +71,10 @@ constexpr int kWarpLoad = 12;   // Q and K tiles
 constexpr int kWarpMma = 13;
 constexpr int kWarpLoadV = 14;  // V tiles
 constexpr uint32_t kTmemCols = 512;
-// setmaxnreg budget: 128 x (168 + 168 + 72 + 104) = 65536 = 512 threads x 128.
-constexpr int kRegsSoftmax = 168;
-constexpr int kRegsEpilogue = 72;
-constexpr int kRegsOther = 104;
+// setmaxnreg budget: 128 x (160 + 160 + 80 + 112) = 65536 = 512 threads x 128.
+constexpr int kRegsSoftmax = 160;
+constexpr int kRegsEpilogue = 80;
+constexpr int kRegsOther = 112;
 static_assert(128 * (2 * kRegsSoftmax + kRegsEpilogue + kRegsOther) == 65536, "register split");
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bit 4),
@@ -94,6 +102,14 @@ struct Params {
   int32_t B, H, Lq, n0, n1;
   int32_t nqp;        // query-tile pairs per (batch, head)
   int32_t num_units;  // B * H * nqp
+  // Tail split: work items [0, head_units) are whole units; the remaining
+  // num_units - head_units units (the last, partial wave) are handed out as
+  // split_k key-range pieces each, so num_items = head_units + (num_units -
+  // head_units) * split_k.  split_k == 1: every item is a whole unit.
+  int32_t head_units, split_k, num_items;
+  uint4* part;         // [slot][tile][4 row quarters][16 chunks][32 rows]: a piece's O / l, 8 bf16 per chunk
+  float2* part_ml;     // [slot][tile][128 rows]: the piece's (row max, row sum)
+  uint32_t* part_cnt;  // [tail unit][tile][4 row quarters]: pieces finished (zeroed by the pre-pass)
   const uint4* table;  // per token 16 x (4 x half2 (cos, sin)): one 16-byte load per 8 dims
   const int32_t* kv_end;
   __nv_bfloat16* o;
@@ -115,6 +131,7 @@ struct __align__(1024) Smem {
   // stages its 32 rows (4 KB) here for its own TMA store
   uint8_t ostage[kHalfBytes];
   float row_l[2][2][BM];  // [unit parity][tile][row]: softmax -> epilogue
+  float row_m[2][2][BM];  // the rows' maxima (read for the pieces of a split unit)
   alignas(16) float qnw[kHeadDim];  // QK-RMSNorm weight of Q (when given)
   int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
   uint64_t q_full[2], q_rot[2], q_empty[2];
@@ -124,6 +141,8 @@ struct __align__(1024) Smem {
   // unit has a single key tile can finish its softmax twice before the
   // epilogue waits; one barrier per unit parity keeps the phases apart
   uint64_t l_ready[2][2];
+  // [tile][epilogue warp]: bulk loads of the pieces to merge after a CTA's last item
+  uint64_t mrg[2][4];
   uint64_t sched_full[kSchedSlots], sched_empty[kSchedSlots];
   uint64_t drain;
   uint32_t tmem_base;
@@ -163,7 +182,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 struct Unit {
   int b, h, row0;
-  int N[2];
+  int N[2];   // key tiles of each query tile in this item
+  int kb;     // first key tile of the item (a piece of a split unit starts past 0)
+  int slot;   // partial-result slot of a piece, -1 for a whole unit
+  int grp;    // tail unit of a piece (its arrival counters)
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -183,6 +205,9 @@ __device__ __forceinline__ int tiles_below(const Params& p, int kv_hi) {
 // workload: 14-15 % faster, the saved DRAM traffic letting the power-capped
 // clock run higher).
 constexpr int kGroup = 16;
+
+// Most pieces a tail unit is split into.
+constexpr int kMaxSplit = 4;
 
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   Unit U;
@@ -214,20 +239,78 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
     const int kv_hi = p.kv_end ? min(p.kv_end[last], p.n0 + p.n1) : p.n0 + p.n1;
     U.N[s] = tiles_below(p, kv_hi);
   }
+  U.kb = 0;
+  U.slot = -1;
+  U.grp = 0;
   return U;
 }
 
-// QK-RMSNorm + rotation of one query row in its 128B-swizzled tile (row t):
-// the row's mean square (fp32, from the bf16 values), then each adjacent pair
-// (2m, 2m+1) scaled by rsqrt(mean square + eps) and the weight and rotated by
-// the token's (cos, sin), rounded once to bf16.
-__device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const uint4* cs, int t,
+// Work item w.  Piece i of a split tail unit covers key tiles
+// [i N / k, (i+1) N / k) of both query tiles; a tail unit whose tiles differ in
+// length or that has fewer than k key tiles goes whole as its piece 0, and its
+// other pieces are empty items (N = 0 for both tiles: every role skips them).
+__device__ __forceinline__ Unit decode_item(const Params& p, int w) {
+  int u = w, g = 0, i = -1;
+  if (w >= p.head_units) {
+    const int j = w - p.head_units;
+    g = j / p.split_k;
+    i = j - g * p.split_k;
+    u = p.head_units + g;
+  }
+  Unit U = decode_unit(p, u);
+  if (i >= 0) {
+    const int N = U.N[0];
+    if (U.N[1] == N && N >= p.split_k) {
+      const int kb = (int)((int64_t)i * N / p.split_k);
+      const int ke = (int)((int64_t)(i + 1) * N / p.split_k);
+      U.kb = kb;
+      U.N[0] = U.N[1] = ke - kb;
+      U.slot = w - p.head_units;
+      U.grp = g;
+    } else if (i > 0) {
+      U.N[0] = U.N[1] = 0;
+    }
+  }
+  return U;
+}
+
+// The token's sixteen 16-byte (cos, sin) chunks (fp16 pairs), all loads in
+// flight at once: one round trip to L2, issued before the query tile lands.
+__device__ __forceinline__ void load_table_row(const uint4* cs, uint4 (&tb)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) tb[i] = __ldg(cs + i);
+}
+
+// Rotation of one query row in its 128B-swizzled tile (row t): each adjacent
+// pair (2m, 2m+1) turned by the token's (cos, sin), rounded once to bf16.
+__device__ __forceinline__ void rotate_q_row(uint8_t* qrow, const uint4 (&tb)[16], int t) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    uint4* ptr = reinterpret_cast<uint4*>(qrow + (c >> 3) * kHalfBytes + (((c & 7) ^ (t & 7)) << 4));
+    uint4 x = *ptr;
+    const __half2* tc = reinterpret_cast<const __half2*>(&tb[c]);
+    uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 xv = unpack_bf16x2(w[e]);
+      const float2 r = __half22float2(tc[e]);  // (cos, sin) of pair 4 c + e
+      w[e] = pack_bf16x2(fmaf(xv.x, r.x, -xv.y * r.y), fmaf(xv.x, r.y, xv.y * r.x));
+    }
+    *ptr = x;
+  }
+}
+
+// QK-RMSNorm + rotation of one query row: the row's mean square (fp32, from
+// the bf16 values), then each adjacent pair (2m, 2m+1) scaled by
+// rsqrt(mean square + eps) and the weight and rotated by the token's
+// (cos, sin), rounded once to bf16.
+__device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const uint4 (&tb)[16], int t,
                                                   const float* wn, float eps) {
   float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll 4
   for (int c = 0; c < 16; ++c) {
-    const int half = c >> 3, cc = c & 7;
-    const uint4 x = *reinterpret_cast<const uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
+    const uint4 x =
+        *reinterpret_cast<const uint4*>(qrow + (c >> 3) * kHalfBytes + (((c & 7) ^ (t & 7)) << 4));
     const uint32_t* w = reinterpret_cast<const uint32_t*>(&x);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -237,16 +320,14 @@ __device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const uint4* cs
     }
   }
   const float rs = rsqrtf((ss0 + ss1) * (1.f / kHeadDim) + eps);
-#pragma unroll 2
+#pragma unroll
   for (int c = 0; c < 16; ++c) {
-    const int half = c >> 3, cc = c & 7;
-    uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((cc ^ (t & 7)) << 4));
+    uint4* ptr = reinterpret_cast<uint4*>(qrow + (c >> 3) * kHalfBytes + (((c & 7) ^ (t & 7)) << 4));
     uint4 x = *ptr;
     const float4 w0 = *reinterpret_cast<const float4*>(wn + 8 * c);
     const float4 w1 = *reinterpret_cast<const float4*>(wn + 8 * c + 4);
     const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    const uint4 tb = __ldg(cs + c);  // the chunk's four (cos, sin) pairs
-    const __half2* tc = reinterpret_cast<const __half2*>(&tb);
+    const __half2* tc = reinterpret_cast<const __half2*>(&tb[c]);
     uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -256,33 +337,6 @@ __device__ __forceinline__ void norm_rotate_q_row(uint8_t* qrow, const uint4* cs
       w[e] = pack_bf16x2(fmaf(x0, r.x, -x1 * r.y), fmaf(x0, r.y, x1 * r.x));
     }
     *ptr = x;
-  }
-}
-
-// Rotation of one query row in its 128B-swizzled tile (row t): each
-// adjacent pair (2m, 2m+1) turned by the token's (cos, sin), rounded once to
-// bf16.  The row's sixteen 16-byte table chunks are loaded in two batches of
-// eight, so the table's latency is paid twice per row, not sixteen times.
-__device__ __forceinline__ void rotate_q_row(uint8_t* qrow, const uint4* cs, int t) {
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint4 tb[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tb[i] = __ldg(cs + 8 * half + i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint4* ptr = reinterpret_cast<uint4*>(qrow + half * kHalfBytes + ((i ^ (t & 7)) << 4));
-      uint4 x = *ptr;
-      const __half2* tc = reinterpret_cast<const __half2*>(&tb[i]);
-      uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 xv = unpack_bf16x2(w[e]);
-        const float2 r = __half22float2(tc[e]);  // (cos, sin) of pair 4 (8 half + i) + e
-        w[e] = pack_bf16x2(fmaf(xv.x, r.x, -xv.y * r.y), fmaf(xv.x, r.y, xv.y * r.x));
-      }
-      *ptr = x;
-    }
   }
 }
 
@@ -383,7 +437,7 @@ __device__ __forceinline__ void publish_unit(Smem& S, const Params& p, uint32_t 
                                   abort, p.status, 0x500));
   if (ok && leader) {
     const uint32_t u = atomicAdd(p.unit_counter, 1u);
-    S.sched_unit[slot] = u < (uint32_t)p.num_units ? (int32_t)u : -1;
+    S.sched_unit[slot] = u < (uint32_t)p.num_items ? (int32_t)u : -1;
     mbar_arrive(smem_u32(&S.sched_full[slot]));
   }
   __syncwarp();
@@ -401,6 +455,77 @@ __device__ __forceinline__ int next_unit(Smem& S, const Params& p, uint32_t& sc,
   }
   ++sc;
   return ok ? u : -1;
+}
+
+// Merge of the k pieces of one warp's 32 rows of a split unit's query tile:
+// O = sum_i a_i (O_i / l_i) with a_i the piece's share of the row sum,
+// a_i = 2^((m_i - M) c) l_i / sum_j 2^((m_j - M) c) l_j, written through the
+// warp's slice of the output stage.  `src` holds the pieces' rows, 8 KB per
+// piece ([16 chunks][32 rows] of 8 bf16) and piece_stride bytes apart, in
+// global memory (read through L2) or, after the CTA's last item, copied into
+// shared memory.
+template <bool kShared>
+__device__ __forceinline__ void merge_pieces(const Params& p, const uint8_t* src, size_t piece_stride,
+                                             const float (&a)[kMaxSplit], uint8_t* stage, int lane, int h,
+                                             int b, int row_first) {
+  for (int hh = 0; hh < 2; ++hh) {
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+#pragma unroll 2
+    for (int ch = 0; ch < 8; ++ch) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kMaxSplit; ++i) {
+        if (i < p.split_k) {
+          const uint4* ptr = reinterpret_cast<const uint4*>(src + i * piece_stride + (8 * hh + ch) * 512) + lane;
+          const uint4 x = kShared ? *ptr : __ldcg(ptr);
+          const uint32_t* xw = reinterpret_cast<const uint32_t*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 v = unpack_bf16x2(xw[e]);
+            acc[2 * e] = fmaf(a[i], v.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(a[i], v.y, acc[2 * e + 1]);
+          }
+        }
+      }
+      *reinterpret_cast<uint4*>(stage + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row_first < p.Lq) {
+      tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, h, row_first, b);
+      bulk_commit_group();
+    }
+    __syncwarp();
+  }
+}
+
+// Shares a_i of the k pieces of row t (see merge_pieces).
+__device__ __forceinline__ void piece_weights(const Params& p, int slot0, int s, int t, float (&a)[kMaxSplit]) {
+  float m[kMaxSplit], l[kMaxSplit];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+    if (i < p.split_k) {
+      const float2 ml = __ldcg(p.part_ml + ((size_t)(slot0 + i) * 2 + s) * BM + t);
+      m[i] = ml.x;
+      l[i] = ml.y;
+      mx = fmaxf(mx, ml.x);
+    }
+  }
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) {
+    a[i] = i < p.split_k ? ex2_approx((m[i] - mx) * kScaleLog2) * l[i] : 0.f;
+    tot += a[i];
+  }
+  const float inv = 1.f / tot;
+#pragma unroll
+  for (int i = 0; i < kMaxSplit; ++i) a[i] *= inv;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
@@ -423,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(smem_u32(&S.o_free[s]), BM);
       mbar_init(smem_u32(&S.l_ready[0][s]), BM);
       mbar_init(smem_u32(&S.l_ready[1][s]), BM);
+      for (int w = 0; w < 4; ++w) mbar_init(smem_u32(&S.mrg[s][w]), 1);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&S.k_full[s]), 1);
@@ -475,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (do_qk) publish_unit(S, p, sc, leader, abort_flag, ok);
         const int u = next_unit(S, p, sc, abort_flag, ok);
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_item(p, u);
         for (int s = 0; s < 2 && ok && do_qk; ++s) {
           if (U.N[s] == 0) continue;
           // the MMA warp releases Q_s once per unit that used it
@@ -493,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         const int N = max(U.N[0], U.N[1]);
         for (int n = 0; n < N && ok; ++n) {
-          const KTile t = key_tile(p, n);
+          const KTile t = key_tile(p, U.kb + n);
           if (do_qk) {
             const int st = kc % kStages;
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_empty[st]), ((kc / kStages) & 1u) ^ 1u,
@@ -555,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       while (ok) {
         const int u = next_unit(S, p, sc, abort_flag, ok);
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_item(p, u);
         const int N = max(U.N[0], U.N[1]);
         if (N == 0) continue;
         // prologue: S_s(0)
@@ -649,53 +775,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       __syncwarp();
     }
   } else if (warp >= kWarpEpi) {
-    // ----------------------------------------------- Q rotation + epilogue
-    // For every unit: rotate its query tiles in place as soon as their TMA
-    // loads land (the MMA warp waits for q_rot before the first S MMA), then
-    // drain the PREVIOUS unit's O.  Rotating first lets the next unit's S
-    // MMAs and softmax start while O of the last unit is still drained.
+    // ------------------------------------------------------------ epilogue
+    // Drains each item's O as soon as its MMAs are done (O / l -> bf16 ->
+    // global, or a piece's partial result), releasing O's TMEM columns for the
+    // next item's first P*V.  The next item is read from the schedule ring
+    // before the drain: the K producer publishes it while this one's keys are
+    // still being loaded, so the read does not delay the drain, and it tells
+    // whether this is the CTA's last item.
     setmaxnreg_dec_epilogue();
     const int t = threadIdx.x & 127;  // row == TMEM lane (warp % 4 picks the lane quarter)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t cnt[2] = {0, 0}, qv[2] = {0, 0}, sc = 0;
-    bool ok = true, have_prev = false;
-    Unit prev;
-    prev.b = prev.h = prev.row0 = 0;
-    prev.N[0] = prev.N[1] = 0;
-    while (ok) {
-      const int u = next_unit(S, p, sc, abort_flag, ok);
+    uint32_t cnt[2] = {0, 0}, sc = 0;
+    bool ok = true;
+    int u = next_unit(S, p, sc, abort_flag, ok);
+    while (ok && u >= 0) {
+      const Unit prev = decode_item(p, u);
+      u = next_unit(S, p, sc, abort_flag, ok);  // -1: prev is the CTA's last item
       if (!ok) break;
-      Unit U;
-      if (u >= 0) {
-        U = decode_unit(p, u);
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (U.N[s] == 0) continue;
-          // the row's 256-byte table row (two 128-byte lines) is pulled into
-          // L1 while the tile's TMA load is still in flight
-          if (U.row0 + s * BM + t < p.Lq) {
-            const uint4* cs = p.table + (size_t)(U.row0 + s * BM + t) * 16;
-            prefetch_l1(cs);
-            prefetch_l1(cs + 8);
-          }
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_full[s]), qv[s] & 1u, abort_flag,
-                                                p.status, 0x300 | s));
-          if (!ok) break;
-          ++qv[s];
-          const int row = U.row0 + s * BM + t;
-          if (row < p.Lq) {
-            const uint4* cs = p.table + (size_t)row * 16;
-            uint8_t* qrow = S.q[s] + t * 128;
-            if (p.q_norm_w == nullptr)
-              rotate_q_row(qrow, cs, t);
-            else
-              norm_rotate_q_row(qrow, cs, t, S.qnw, p.norm_eps);
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(smem_u32(&S.q_rot[s]));
-        }
-        if (!ok) break;
-      }
-      for (int s = 0; s < 2 && ok && have_prev; ++s) {
+      bool merge_pending[2] = {false, false};
+      for (int s = 0; s < 2 && ok; ++s) {
         if (prev.N[s] == 0) continue;
         const uint32_t par = cnt[s] & 1u;
         const uint32_t lpar = (cnt[s] >> 1) & 1u;  // phase of l_ready[par][s]
@@ -707,24 +805,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                               p.status, 0x410 | s));
         if (!ok) break;
         tc_fence_after();
-        const float inv = 1.f / S.row_l[par][s][t];
         const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
-        // O / l -> bf16 in two 64-column halves.  Each warp stages its own 32
-        // rows in shared memory (128B-swizzled, the TMA layout) and writes
-        // them with one TMA store (rows past Lq are clipped; a box wholly past
-        // Lq is not issued).  O's TMEM columns are released as soon as the
-        // second half has been read, long before the stores finish.  No
-        // barrier spans warps, so a warp that gives up on a timed-out wait
-        // cannot hold the others.
         uint8_t* stage = S.ostage + (warp & 3) * 32 * 128;
         const int row_first = prev.row0 + s * BM + (warp & 3) * 32;
-        for (int hh = 0; hh < 2; ++hh) {
-          if (lane == 0) bulk_wait_read_all();  // this warp's slice of the stage is free
-          __syncwarp();
+        if (prev.slot < 0) {
+          // O / l -> bf16 in two 64-column halves.  Each warp stages its own
+          // 32 rows in shared memory (128B-swizzled, the TMA layout) and
+          // writes them with one TMA store (rows past Lq are clipped; a box
+          // wholly past Lq is not issued).  O's TMEM columns are released as
+          // soon as the second half has been read, long before the stores
+          // finish.  No barrier spans warps, so a warp that gives up on a
+          // timed-out wait cannot hold the others.
+          const float inv = 1.f / S.row_l[par][s][t];
+          for (int hh = 0; hh < 2; ++hh) {
+            if (lane == 0) bulk_wait_read_all();  // this warp's slice of the stage is free
+            __syncwarp();
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2; ++c) {
+              uint32_t orow[32];
+              tmem_ld32(tO + 64 * hh + 32 * c, orow);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
+                                     __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
+                const int chunk = 4 * c + e;  // 16-byte chunk of the 128-byte row
+                *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+            if (hh == 1) {
+              tc_fence_before();
+              mbar_arrive(smem_u32(&S.o_free[s]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row_first < p.Lq) {
+              tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, prev.h, row_first, prev.b);
+              bulk_commit_group();
+            }
+            __syncwarp();
+          }
+          continue;
+        }
+        // A piece of a split unit: its O / l (bf16) and (row max, row sum)
+        // go to the piece's slot; the warp that finishes the last piece of
+        // these 32 rows merges all pieces.  Nothing waits for another CTA:
+        // the arrival counter decides who merges.
+        const size_t part_off = (((size_t)prev.slot * 2 + s) * 4 + (warp & 3)) * 8192;  // bytes
+        {
+          const float l = S.row_l[par][s][t];
+          const float m = S.row_m[par][s][t];
+          const float inv = 1.f / l;
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.part) + part_off) + lane;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
             uint32_t orow[32];
-            tmem_ld32(tO + 64 * hh + 32 * c, orow);
+            tmem_ld32(tO + 32 * c, orow);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -733,27 +873,67 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               for (int i = 0; i < 4; ++i)
                 w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
                                    __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
-              const int chunk = 4 * c + e;  // 16-byte chunk of the 128-byte row
-              *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
+              dst[(4 * c + e) * 32] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
-          if (hh == 1) {
-            tc_fence_before();
-            mbar_arrive(smem_u32(&S.o_free[s]));
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row_first < p.Lq) {
-            tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, prev.h, row_first, prev.b);
-            bulk_commit_group();
-          }
-          __syncwarp();
+          tc_fence_before();
+          mbar_arrive(smem_u32(&S.o_free[s]));
+          p.part_ml[(size_t)(prev.slot * 2 + s) * BM + t] = make_float2(m, l);
+        }
+        __threadfence();
+        __syncwarp();
+        uint32_t arrived = 0;
+        if (lane == 0) arrived = atomicAdd(p.part_cnt + ((size_t)prev.grp * 2 + s) * 4 + (warp & 3), 1u);
+        arrived = __shfl_sync(0xffffffffu, arrived, 0);
+        if (arrived != (uint32_t)(p.split_k - 1)) continue;
+        __syncwarp();
+        __threadfence();
+        if (u < 0) {
+          // the CTA's last item: merged below, once both tiles' MMAs are done
+          merge_pending[s] = true;
+          continue;
+        }
+        {
+          float a[kMaxSplit];
+          const int slot0 = prev.grp * p.split_k;
+          piece_weights(p, slot0, s, t, a);
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(p.part) +
+                               (((size_t)slot0 * 2 + s) * 4 + (warp & 3)) * 8192;
+          // consecutive slots are 2 tiles x 4 row quarters x 8 KB apart
+          merge_pieces<false>(p, src, 65536, a, stage, lane, prev.h, prev.b, row_first);
         }
       }
-      if (u < 0) break;
-      prev = U;
-      have_prev = true;
+      if (u < 0) {
+        // Merges that fell to this warp on the CTA's last item.  Every MMA of
+        // the CTA has completed (both tiles' o_done were waited above) and no
+        // load is in flight, so the Q and K buffers are free: each warp bulk-
+        // loads its rows of the k pieces (8 KB each) into its 32 KB of them,
+        // one round trip instead of one per 16-byte chunk.
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!merge_pending[s]) continue;
+          float a[kMaxSplit];
+          const int slot0 = prev.grp * p.split_k;
+          piece_weights(p, slot0, s, t, a);
+          uint8_t* buf = S.q[0] + (warp & 3) * 32768;
+          const uint32_t bar = smem_u32(&S.mrg[s][warp & 3]);
+          fence_proxy_async_smem();  // earlier reads of buf come before the copies
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)p.split_k * 8192u);
+            for (int i = 0; i < p.split_k; ++i)
+              bulk_load(smem_u32(buf) + i * 8192,
+                        reinterpret_cast<const uint8_t*>(p.part) +
+                            (((size_t)(slot0 + i) * 2 + s) * 4 + (warp & 3)) * 8192,
+                        8192u, bar);
+          }
+          __syncwarp();
+          ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, abort_flag, p.status, 0x420 | s));
+          if (!ok) break;
+          merge_pieces<true>(p, buf, 8192, a, S.ostage + (warp & 3) * 32 * 128, lane, prev.h, prev.b,
+                             prev.row0 + s * BM + (warp & 3) * 32);
+        }
+        break;
+      }
     }
     // the shared-memory stage must stay valid until the last stores read it
     if (lane == 0) bulk_wait_read_all();
@@ -766,18 +946,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + s * BN;
     const uint32_t tO = tmem + lane_base + 256 + s * kHeadDim;
-    uint32_t uc = 0, sf = 0, sc = 0;
+    uint32_t uc = 0, sf = 0, sc = 0, qv = 0;
     bool ok = true;
     while (ok) {
       const int u = next_unit(S, p, sc, abort_flag, ok);
       if (u < 0) break;
-      const Unit U = decode_unit(p, u);
+      const Unit U = decode_item(p, u);
       const int Ns = U.N[s];
       if (Ns == 0) continue;
       const int row = U.row0 + s * BM + t;
       const bool valid = row < p.Lq;
       const uint32_t par = uc & 1u;  // unit parity of this tile's l buffer
       ++uc;
+      {
+        // Rotate this thread's query row in place once the tile's TMA load
+        // lands (the MMA warp waits for q_rot before the first S MMA).  The
+        // group is idle here (its last tile of the previous item is done),
+        // and the row's table chunks are requested before the wait (rows
+        // past Lq read the last row's and leave their zero-filled Q alone).
+        uint4 tb[16];
+        load_table_row(p.table + (size_t)min(row, p.Lq - 1) * 16, tb);
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.q_full[s]), qv & 1u, abort_flag, p.status,
+                                              0x300 | s));
+        if (!ok) break;
+        ++qv;
+        if (valid) {
+          uint8_t* qrow = S.q[s] + t * 128;
+          if (p.q_norm_w == nullptr)
+            rotate_q_row(qrow, tb, t);
+          else
+            norm_rotate_q_row(qrow, tb, t, S.qnw, p.norm_eps);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&S.q_rot[s]));
+      }
       const int kv_i = valid ? (p.kv_end ? p.kv_end[row] : p.n0 + p.n1) : p.n0 + p.n1;
       float m = -INFINITY, l = 0.f;
       for (int n = 0; n < Ns; ++n) {
@@ -793,7 +995,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tmem_wait_ld();
         float* sv = reinterpret_cast<float*>(sr);
-        const KTile kt = key_tile(p, n);
+        const KTile kt = key_tile(p, U.kb + n);
         const int lim = max(0, min(kt.cnt, kv_i - kt.j0));
         const bool masked = __any_sync(0xffffffffu, lim < BN);
         float alpha = 1.f, mc;
@@ -844,6 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       if (!ok) break;
       S.row_l[par][s][t] = l;
+      S.row_m[par][s][t] = m;
       mbar_arrive(smem_u32(&S.l_ready[par][s]));
     }
   }
@@ -901,6 +1104,10 @@ static bool encode_source(CUtensorMap* m, const KvSource& s, int B, int H, int* 
   return encode_4d(m, s.ptr, s.n, H, B, s.row * e, s.head * e, s.batch * e, tc::BM, 1);
 }
 
+// Tail-split cost model constants (key tiles), see launch_attn_tc_bf16.
+constexpr float kSplitItemTiles = 3.5f;
+constexpr float kSplitMergeTiles = 9.0f;
+
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms) {
   if (a.Lq == 0 || a.B == 0 || a.H == 0) return cudaSuccess;
   tc::Params p;
@@ -928,11 +1135,42 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.unit_counter = a.unit_counter;
   p.q_norm_w = a.q_norm_w;
   p.norm_eps = a.norm_eps;
+  // Tail split (unmasked calls, where every unit visits the same key tiles):
+  // the r units of the last, partial wave go out as k pieces each when that
+  // shortens the wave.  Costs in key tiles of one unit, from per-CTA
+  // timelines: each item start (Q load and rotation, the first tiles' fill)
+  // about 3.5; the merge the last CTA cannot overlap, plus the slowdown of
+  // the whole units running beside the pieces, about 9 (with these the
+  // 384-unit 1024^2 step, 34 key tiles per unit, stays unsplit: split into 3
+  // it measured 3 % slower).
+  p.head_units = p.num_units;
+  p.split_k = 1;
+  if (a.kv_end == nullptr && a.split_slots > 0 && num_sms > 0) {
+    const int r = p.num_units % num_sms;
+    const int N = (p.n0 + tc::BN - 1) / tc::BN + (p.n1 + tc::BN - 1) / tc::BN;
+    if (r > 0 && r <= a.split_cnt_units) {
+      float best = (float)N + kSplitItemTiles;
+      for (int k = 2; k <= tc::kMaxSplit; ++k) {
+        if (N < k || r * k > a.split_slots) break;
+        const float cost = (float)((r * k + num_sms - 1) / num_sms) * ((float)N / k + kSplitItemTiles) +
+                           kSplitMergeTiles;
+        if (cost < best) {
+          best = cost;
+          p.split_k = k;
+        }
+      }
+      if (p.split_k > 1) p.head_units = p.num_units - r;
+    }
+  }
+  p.num_items = p.head_units + (p.num_units - p.head_units) * p.split_k;
+  p.part = static_cast<uint4*>(a.split_part);
+  p.part_ml = static_cast<float2*>(a.split_ml);
+  p.part_cnt = a.split_cnt;
   const size_t smem = sizeof(tc::Smem) + 1024;
   cudaError_t err =
       cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  const int grid = p.num_items < num_sms ? p.num_items : num_sms;
   tc::attn_tc_kernel<<<grid, tc::kThreads, smem, stream>>>(p);
   note_launch();
   return cudaGetLastError();

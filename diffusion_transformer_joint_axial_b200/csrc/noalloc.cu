@@ -42,7 +42,7 @@ extern "C" qi21_status qi21_attn_cached_noalloc(int32_t B, int32_t H, int64_t P,
                                                 const void* v, const int32_t* pos_tgt,
                                                 const void* k_cache, const void* v_cache, void* o,
                                                 void* stream) {
-  const size_t need = qi21_attn_cached_workspace_size(B, H, P, T, dt);
+  const size_t need = qi21::attn_cached_workspace_min(B, H, T, dt);
   if (need > kNoAllocScratchBytes)
     return qi21::report_error(
         QI21_ERR_INVALID_ARG,

@@ -174,8 +174,10 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int H = p.H;
   const bool has_tok = tok < p.Lk;
   const int iters = (H + SPT - 1) / SPT;  // the same for every thread (shuffle reductions)
-  if (p.unit_counter != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
-    *p.unit_counter = 0u;
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    if (p.unit_counter != nullptr && threadIdx.x == 0) *p.unit_counter = 0u;
+    for (int i = threadIdx.x; i < p.n_zero_words; i += blockDim.x) p.zero_words[i] = 0u;
+  }
   const bool norm = p.k_norm_w != nullptr;
   const T* __restrict__ kp = static_cast<const T*>(p.k) + ((static_cast<int64_t>(b) * p.Lk + tok) * H) *
                                                               kHeadDim + c * EPC;

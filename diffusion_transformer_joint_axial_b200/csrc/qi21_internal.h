@@ -61,6 +61,8 @@ struct RopePrepParams {
   void* table;     // [Lk][64] (cos, sin) of every token, or null: float2, or half2 when table_half
   int32_t table_half;
   uint32_t* unit_counter;  // zeroed here for the attention launch that follows, or null
+  uint32_t* zero_words;    // also zeroed here (the attention's tail-split counters), or null
+  int32_t n_zero_words;
   Omega omega;
   const float* k_norm_w;   // [128] QK-RMSNorm weight of K, or null (no norm)
   float norm_eps;
@@ -91,6 +93,16 @@ struct AttnArgs {
   uint32_t* unit_counter; // workspace header: dynamic-schedule counter (zeroed by the pre-pass)
   const float* q_norm_w;  // [128] QK-RMSNorm weight of Q, or null (no norm)
   float norm_eps;
+  // Scratch for splitting the last, partial wave of units into key-range
+  // pieces (unmasked calls only; null / 0: no split).  split_cnt holds
+  // split_cnt_units x 8 arrival counters, zeroed by the pre-pass; split_part
+  // and split_ml hold the O / l (bf16) and (row max, row sum) of up to
+  // split_slots pieces.  The launcher decides how many pieces it uses.
+  uint32_t* split_cnt;
+  int32_t split_cnt_units;
+  void* split_part;   // split_slots x 2 tiles x 128 rows x 128 bf16
+  void* split_ml;     // split_slots x 2 tiles x 128 rows x float2
+  int32_t split_slots;
 };
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);
@@ -122,6 +134,11 @@ cudaError_t launch_swiglu(int64_t n, const void* g, const void* u, void* m, cuda
 
 // --------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+// Bytes a cached step needs at least (no tail-split scratch);
+// qi21_attn_cached_workspace_size() adds the scratch that lets the last wave
+// of units be split.
+size_t attn_cached_workspace_min(int32_t B, int32_t H, int64_t T, qi21_dtype dt);
 
 // Device address of qi21_attn_cached_noalloc's built-in scratch on the
 // current device (noalloc.cu).

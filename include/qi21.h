@@ -152,7 +152,13 @@ qi21_status qi21_attn_full(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtyp
                            void* k_cache, void* v_cache,
                            void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes qi21_attn_cached needs for these sizes (header included). */
+/* Workspace bytes for qi21_attn_cached with these sizes (header included).
+ * For bf16 this includes scratch for splitting the last, partial wave of
+ * work units into key-range pieces (up to 512 pieces of 66 KB, and arrival
+ * counters); a smaller workspace still works as long as it holds the table
+ * and the rotated target keys -- the call then splits fewer units or none
+ * (the no-allocation entry point below runs that way when its 32 MiB are
+ * short). */
 size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt);
 
 /*
@@ -285,7 +291,9 @@ qi21_status qi21_swiglu(int64_t n, const void* g, const void* u, void* m, void* 
  * Same arguments and result as qi21_attn_cached minus the workspace: the
  * scratch is a 32 MiB array built into the library, held by every GPU that
  * loads the library until the process exits.  Calls needing more than that
- * (qi21_attn_cached_workspace_size() > 32 MiB) return QI21_ERR_INVALID_ARG
+ * (more than 32 MiB for the position table and the rotated target keys, about
+ * B * H * T * 256 bytes + T * 512 bytes; the 2048^2 workload's cached step
+ * needs ~200 MB) return QI21_ERR_INVALID_ARG
  * without enqueuing anything; so does every other argument error.  Each call
  * looks up the array's device address on the current device; the first call
  * on a device also loads the library's device code there, so make it before
