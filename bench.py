@@ -42,12 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # pre-pass plus the attention kernel -- from one ncu capture of each kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum), per workload.  Valid only for
 # the kernel sources they were taken on: any other source reports null.
-NCU_TRAFFIC = {"sources_sha256": "c29186fd2ac63ae9",
+NCU_TRAFFIC = {"sources_sha256": "5ac1f16f98ba228e",
                # mean of the full and the cached call
-               "bytes_per_call": {"t2i": ((28.398e6 + 0.049e6 + 82.029e6 + 1.389e6)
-                                          + (25.249e6 + 0.000e6 + 79.810e6 + 0.573e6)) / 2,
-                                  "hires": ((315.109e6 + 262.659e6 + 2619.034e6 + 250.149e6)
-                                            + (201.724e6 + 144.889e6 + 2426.388e6 + 208.678e6)) / 2}}
+               "bytes_per_call": {"t2i": ((28.399e6 + 0.056e6 + 82.075e6 + 2.679e6)
+                                          + (25.249e6 + 0.002e6 + 79.889e6 + 1.773e6)) / 2,
+                                  "hires": ((315.143e6 + 261.812e6 + 2601.413e6 + 277.252e6)
+                                            + (201.800e6 + 145.300e6 + 2430.348e6 + 235.585e6)) / 2}}
 
 
 def kernel_sources_digest(read=None):
