@@ -374,20 +374,29 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, int tok_maj
 
 // The start-address field of a descriptor is (address >> 4) in its low 14
 // bits; shared-memory addresses stay below 256 KB, so moving a descriptor by a
-// byte offset is one 64-bit add of offset >> 4 that never carries out of the
-// field.
+// byte offset is a 32-bit add of offset >> 4 to its low word that never
+// carries out of the field.  The MMA warp shares an SMSP with two softmax
+// warps, which then reach their barriers last: every instruction it saves
+// (this add, the per-stage descriptors built once) shortens the step
+// (measured 1-2 % on every workload).
+__device__ __forceinline__ uint64_t desc_lo_add(uint64_t d, uint32_t off) {
+  const uint32_t lo = (uint32_t)d + off, hi = (uint32_t)(d >> 32);
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t qdesc, uint64_t kdesc) {
 #pragma unroll
   for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-    const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
-    mma_ss(tmem_s, qdesc + off, kdesc + off, kIdescS, kk > 0);
+    const uint32_t off = (uint32_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+    mma_ss(tmem_s, desc_lo_add(qdesc, off), desc_lo_add(kdesc, off), kIdescS, kk > 0);
   }
 }
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t vdesc, int kk0,
                                          bool first) {
 #pragma unroll
   for (int kk = kk0; kk < kk0 + 4; ++kk)
-    mma_ts(tmem_o, tmem_p + kk * 8, vdesc + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+    mma_ts(tmem_o, tmem_p + kk * 8, desc_lo_add(vdesc, (uint32_t)((kk * 2048) >> 4)), kIdescPV,
            (!first || kk > 0) ? 1u : 0u);
 }
 
@@ -672,6 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const bool leader = elect_one_sync();
       const uint64_t qdesc[2] = {sw128_desc(smem_u32(S.q[0]), 16, 1024),
                                  sw128_desc(smem_u32(S.q[1]), 16, 1024)};
+      const uint64_t kdesc0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);
+      const uint64_t kdesc1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
+      const uint64_t vdesc0 = sw128_desc(smem_u32(S.v[0]), kHalfBytes, 1024);
+      const uint64_t vdesc1 = sw128_desc(smem_u32(S.v[1]), kHalfBytes, 1024);
       uint32_t kc = 0, vc = 0, qv[2] = {0, 0}, ph[2] = {0, 0}, pf[2] = {0, 0}, of[2] = {0, 0};
       bool ok = true;
       auto wait = [&](uint64_t& bar, uint32_t parity, uint32_t where) {
@@ -690,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = wait(S.k_full[st], (kc / kStages) & 1u, 0x210);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t kdesc = sw128_desc(smem_u32(S.k[st]), 16, 1024);
+          const uint64_t kdesc = st ? kdesc1 : kdesc0;
           for (int s = 0; s < 2 && ok; ++s) {
             if (U.N[s] == 0) continue;
             ok = wait(S.q_rot[s], qv[s] & 1u, 0x220 | s);
@@ -714,9 +727,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = wait(S.v_full[vst], (vc / kStages) & 1u, 0x230 | vst);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t vdesc = sw128_desc(smem_u32(S.v[vst]), kHalfBytes, 1024);
+          const uint64_t vdesc = vst ? vdesc1 : vdesc0;
           const int kst = kc % kStages;
-          const uint64_t kdesc = sw128_desc(smem_u32(S.k[kst]), 16, 1024);
+          const uint64_t kdesc = kst ? kdesc1 : kdesc0;
           bool k_ready = false;
           for (int s = 0; s < 2 && ok; ++s) {
             const uint32_t tS = tmem + s * BN;
