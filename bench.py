@@ -509,6 +509,8 @@ def bench_workload(qi, args, name, world, dev, flush, clocks, headline):
     else:
         full_fn, cached_fn = lib.qi21_attn_full, lib.qi21_attn_cached
     positions_fn = lib.qi21_rope_positions_original if orig else lib.qi21_rope_positions
+    # the earlier model attends without a mask: kv_end NULL (every key visible)
+    kv_arg = None if orig else kv_end
 
     def one_step(ev=None):
         if ev is not None:
@@ -517,7 +519,7 @@ def bench_workload(qi, args, name, world, dev, flush, clocks, headline):
         assert st == 0, lib.qi21_last_error()
         if ev is not None:
             ev[1].record(stream)
-        st = full_fn(B, H, L, 0 if orig else P, 0, P_(dq), P_(dk), P_(dv), P_(pos), P_(kv_end), P_(o_full),
+        st = full_fn(B, H, L, 0 if orig else P, 0, P_(dq), P_(dk), P_(dv), P_(pos), P_(kv_arg), P_(o_full),
                      P_(kc), P_(vc), P_(ws_f), ws_f.numel(), sp)
         assert st == 0, lib.qi21_last_error()
         if ev is not None:
@@ -623,7 +625,7 @@ def bench_workload(qi, args, name, world, dev, flush, clocks, headline):
             spn = qi._binding.ctypes.c_void_p(stream.cuda_stream)
             st = positions_fn(seg_arr, len(segs), L, P_(pos), P_(kv_end), spn)
             assert st == 0, lib.qi21_last_error()
-            st = full_fn(B, H, L, 0 if orig else P, 0, P_(d_in[0]), P_(d_in[1]), P_(d_in[2]), P_(pos), P_(kv_end),
+            st = full_fn(B, H, L, 0 if orig else P, 0, P_(d_in[0]), P_(d_in[1]), P_(d_in[2]), P_(pos), P_(kv_arg),
                          P_(d_out[0]), P_(kc), P_(vc), P_(ws_f), ws_f.numel(), spn)
             assert st == 0, lib.qi21_last_error()
             full_done = ev()

@@ -215,7 +215,8 @@ def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=
     """First step: block-causal joint attention; stores the prefix K/V cache if given.
 
     q, k, v: [B, L, H, 128] bf16 or fp32 on one CUDA device; pos [L, 3],
-    kv_end [L] int32 from :func:`rope_positions`.  ``qk_norm = (w_q, w_k, eps)``
+    kv_end [L] int32 from :func:`rope_positions`, or None for no mask (every
+    query sees all L keys, as in the earlier model).  ``qk_norm = (w_q, w_k, eps)``
     (float32 [128] weights on the same device) fuses the QK-RMSNorm in front of
     the rotation.  Returns ``out``.
     """
@@ -226,7 +227,8 @@ def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, (B, L, H, HEAD_DIM), dt, dev)
     _need(pos, "pos", (L, 3), torch.int32, dev)
-    _need(kv_end, "kv_end", (L,), torch.int32, dev)
+    if kv_end is not None:
+        _need(kv_end, "kv_end", (L,), torch.int32, dev)
     P = int(prefix_len)
     if out is None:
         out = torch.empty_like(q)

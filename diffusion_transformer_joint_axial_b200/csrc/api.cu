@@ -76,6 +76,31 @@ static SplitCaps split_caps(int64_t B, int64_t H, int64_t T) {
   return c;
 }
 
+// Bytes of the tail-split scratch for a call over `rows` query rows (bf16).
+static size_t split_bytes(int64_t B, int64_t H, int64_t rows) {
+  const SplitCaps c = split_caps(B, H, rows);
+  return c.cnt_bytes + (size_t)c.slots * (kSplitSlotPartBytes + kSplitSlotMlBytes);
+}
+
+// Hands the attention the tail-split scratch that the workspace holds past
+// its minimum layout (none: the call runs unsplit); the pre-pass zeroes the
+// arrival counters.
+static void carve_split(AttnArgs& a, RopePrepParams& rp, uint8_t* ws, size_t base, size_t workspace_bytes,
+                        int64_t B, int64_t H, int64_t rows) {
+  const SplitCaps c = split_caps(B, H, rows);
+  const size_t avail = workspace_bytes - base;
+  if (avail < c.cnt_bytes + kSplitSlotPartBytes + kSplitSlotMlBytes) return;
+  int64_t slots = (int64_t)((avail - c.cnt_bytes) / (kSplitSlotPartBytes + kSplitSlotMlBytes));
+  if (slots > c.slots) slots = c.slots;
+  a.split_cnt = reinterpret_cast<uint32_t*>(ws + base);
+  a.split_cnt_units = (int32_t)c.units;
+  a.split_part = ws + base + c.cnt_bytes;
+  a.split_ml = ws + base + c.cnt_bytes + (size_t)slots * kSplitSlotPartBytes;
+  a.split_slots = (int32_t)slots;
+  rp.zero_words = a.split_cnt;
+  rp.n_zero_words = (int32_t)(c.units * 8);
+}
+
 static int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -197,7 +222,9 @@ qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_seg
 
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt) {
   if (B < 0 || H < 0 || L < 0 || P < 0 || P > L) return 0;
-  return ws_layout(B, H, L, L - P, dt).total;
+  const size_t base = ws_layout(B, H, L, L - P, dt).total;
+  if (dt != QI21_BF16 || B == 0 || H == 0 || L == 0) return base;
+  return base + split_bytes(B, H, L);
 }
 
 size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt) {
@@ -205,8 +232,7 @@ size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t 
   if (B < 0 || H < 0 || T < 0) return 0;
   const size_t base = ws_layout(B, H, T, T, dt).total;
   if (dt != QI21_BF16 || B == 0 || H == 0 || T == 0) return base;
-  const SplitCaps c = split_caps(B, H, T);
-  return base + c.cnt_bytes + (size_t)c.slots * (kSplitSlotPartBytes + kSplitSlotMlBytes);
+  return base + split_bytes(B, H, T);
 }
 
 static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
@@ -225,7 +251,7 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   QI21_TRY(check_ptr(v, "v"));
   QI21_TRY(check_ptr(o, "o"));
   QI21_TRY(check_ptr(pos, "pos"));
-  QI21_TRY(check_ptr(kv_end, "kv_end"));
+  if (kv_end != nullptr) QI21_TRY(check_ptr(kv_end, "kv_end"));
   if (k_cache != nullptr && P > 0) {
     QI21_TRY(check_ptr(k_cache, "k_cache"));
     QI21_TRY(check_ptr(v_cache, "v_cache"));
@@ -263,12 +289,14 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;
   rp.norm_eps = eps;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  // without a mask every unit costs the same, so the last wave may be split
+  if (dt == QI21_BF16 && kv_end == nullptr) carve_split(a, rp, ws, w.total, workspace_bytes, B, H, L);
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
   const int64_t tokstride = (int64_t)H * kHeadDim;
-  AttnArgs a;
-  memset(&a, 0, sizeof(a));
   a.unit_counter = rp.unit_counter;
   a.B = B;
   a.H = H;
@@ -344,21 +372,7 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   // (none: the call runs unsplit).
   AttnArgs a;
   memset(&a, 0, sizeof(a));
-  if (dt == QI21_BF16) {
-    const SplitCaps c = split_caps(B, H, T);
-    const size_t avail = workspace_bytes - w.total;
-    if (avail >= c.cnt_bytes + kSplitSlotPartBytes + kSplitSlotMlBytes) {
-      int64_t slots = (int64_t)((avail - c.cnt_bytes) / (kSplitSlotPartBytes + kSplitSlotMlBytes));
-      if (slots > c.slots) slots = c.slots;
-      a.split_cnt = reinterpret_cast<uint32_t*>(ws + w.total);
-      a.split_cnt_units = (int32_t)c.units;
-      a.split_part = ws + w.total + c.cnt_bytes;
-      a.split_ml = ws + w.total + c.cnt_bytes + (size_t)slots * kSplitSlotPartBytes;
-      a.split_slots = (int32_t)slots;
-      rp.zero_words = a.split_cnt;
-      rp.n_zero_words = (int32_t)(c.units * 8);
-    }
-  }
+  if (dt == QI21_BF16) carve_split(a, rp, ws, w.total, workspace_bytes, B, H, T);
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 

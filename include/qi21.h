@@ -111,10 +111,13 @@ qi21_status qi21_rope_positions(const qi21_segment* segs, int32_t n_segs, int64_
 qi21_status qi21_rope_positions_original(const qi21_segment* segs, int32_t n_segs, int64_t L,
                                          int32_t* pos, int32_t* kv_end, void* stream);
 
-/* Workspace bytes qi21_attn_full needs for these sizes (header included).
+/* Workspace bytes for qi21_attn_full with these sizes (header included).
  * P is the number of rows the call will store in a cache: pass the prefix
  * length when k_cache/v_cache are given and 0 when they are not (the call
- * checks workspace_bytes against the size for the rows it keeps). */
+ * checks workspace_bytes against the size for the rows it keeps).  For bf16
+ * it includes the scratch for splitting the last wave of work units, used
+ * only by calls without a mask (kv_end NULL); a workspace without it (the
+ * table and the rotated keys) still works. */
 size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt);
 
 /*
@@ -135,7 +138,10 @@ size_t qi21_attn_full_workspace_size(int32_t B, int32_t H, int64_t L, int64_t P,
  *   pos         device int32 [L][3] from qi21_rope_positions.
  *   kv_end      device int32 [L] from qi21_rope_positions; must be
  *               non-decreasing with 1 <= kv_end[i] <= L (the builder's output
- *               always is).
+ *               always is).  NULL: no mask, every query sees all L keys (the
+ *               earlier model's layout, where qi21_rope_positions_original
+ *               writes kv_end = L); such a call may also split its last,
+ *               partial wave of work units like qi21_attn_cached.
  *   o           device [B, L, H, 128], written.
  *   k_cache     device [B, H, P, 128] or NULL: rotated prefix K, written.
  *   v_cache     device [B, H, P, 128] or NULL: prefix V, written (both or

@@ -48,17 +48,29 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
+    rnd = lambda x: (x + 255) // 256 * 256
+
+    def split_region(B, H, rows):
+        # tail-split scratch: arrival counters of up to 512 units, then up to
+        # 512 piece slots of 64 KB (O / l) + 2 KB (row max, row sum)
+        units = B * H * ((rows + 255) // 256)
+        return rnd(min(units, 512) * 8 * 4) + min(4 * units, 512) * (65536 + 2048)
+
+    def base(B, H, table_rows, k_rows):
+        # header + cos/sin table (rows x 64 float2) + rotated keys of the rows
+        # not stored in a cache (B x H x k_rows x 128 bf16)
+        return rnd(rnd(256 + table_rows * 64 * 8) + B * H * k_rows * 128 * 2)
+
     full = lib.qi21_attn_full_workspace_size(1, 24, 4352, 256, qb.QI21_BF16)
-    # header + cos/sin table (L x 64 float2) + rotated keys of the rows not
-    # stored in the cache (B x H x (L - P) x 128 bf16)
-    assert full >= 256 + 4352 * 64 * 8 + 24 * 4096 * 128 * 2
-    assert full < 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
+    assert full == base(1, 24, 4352, 4096) + split_region(1, 24, 4352)
     assert full % 256 == 0
     no_cache = lib.qi21_attn_full_workspace_size(1, 24, 4352, 0, qb.QI21_BF16)
-    assert no_cache >= 256 + 4352 * 64 * 8 + 24 * 4352 * 128 * 2
+    assert no_cache == base(1, 24, 4352, 4352) + split_region(1, 24, 4352)
+    f32 = lib.qi21_attn_full_workspace_size(1, 2, 300, 0, qb.QI21_F32)
+    assert f32 == rnd(rnd(256 + 300 * 64 * 8) + 2 * 300 * 128 * 4)  # fp32: no split scratch
     assert lib.qi21_attn_full_workspace_size(1, 24, 4352, 4353, qb.QI21_BF16) == 0  # P > L
     cached = lib.qi21_attn_cached_workspace_size(1, 24, 256, 4096, qb.QI21_BF16)
-    assert cached >= 256 + 4096 * 64 * 8 + 24 * 4096 * 128 * 2
+    assert cached == base(1, 24, 4096, 4096) + split_region(1, 24, 4096)
     assert lib.qi21_attn_full_workspace_size(-1, 1, 1, 0, 0) == 0
 
 

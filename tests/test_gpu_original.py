@@ -65,3 +65,46 @@ def test_original_workload_full_size_sampled(cuda_device):
     hs = [0, 12, 23]
     ref = O.attn_full(*(W.as_f64(x[:, :, hs]) for x in (q, k, v)), opos, okv, rows=rows)
     assert_close(got[:, rows][:, :, hs], ref, torch.bfloat16, "orig full (sampled)")
+
+
+def _full_unmasked(segs, q, k, v, dev):
+    """The same call with kv_end = NULL (no mask): the launcher may split the
+    last wave of units into key-range pieces."""
+    B, L, H, _ = q.shape
+    pos, _ = qi.rope_positions(segs, dev, original=True)
+    ws = qi.new_workspace(qi.full_workspace_size(B, H, L, 0, q.dtype), dev)
+    o = qi.attn_full(q.to(dev), k.to(dev), v.to(dev), pos, None, 0, workspace=ws)
+    check_status(ws)
+    torch.cuda.synchronize()
+    return o.cpu()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("name", ["edit_small", "odd", "split_4"])
+def test_original_without_kv_end(cuda_device, name, dtype):
+    """kv_end NULL means every key is visible: the oracle's unmasked result.
+    split_4 (32 units of 16 key tiles) is split into 4 pieces per unit."""
+    segs = LAYOUTS[name] if name in LAYOUTS else [T_(256), I_(32, 32, 0), I_(24, 32, 1)]
+    L = sum(W.seg_tokens(s) for s in segs)
+    B, H = (1, 4) if name == "split_4" else (2, 3)
+    q, k, v = W.draw_qkv(B, L, H, 29, "bf16" if dtype == torch.bfloat16 else "f32")
+    got = _full_unmasked(segs, q, k, v, cuda_device)
+    opos, okv = O.positions_original(segs)
+    ref = O.attn_full(W.as_f64(q), W.as_f64(k), W.as_f64(v), opos, okv)
+    assert_close(got, ref, dtype, "original without kv_end " + name)
+
+
+def test_original_workload_full_size_without_kv_end(cuda_device):
+    """The earlier model's full workload with kv_end NULL (its last wave is
+    split into 3 pieces per unit on a 148-SM B200), sampled rows including the
+    rows of the split units (rows 0-255 of every head)."""
+    name = "orig"
+    cfg = W.WORKLOADS[name]
+    L = sum(W.seg_tokens(s) for s in cfg["segments"])
+    q, k, v = W.full_inputs(name)
+    got = _full_unmasked(cfg["segments"], q, k, v, cuda_device)
+    opos, okv = O.positions_original(cfg["segments"])
+    rows = sample_rows(L, 256, okv, np.random.default_rng(8))
+    hs = [0, 12, 23]
+    ref = O.attn_full(*(W.as_f64(x[:, :, hs]) for x in (q, k, v)), opos, okv, rows=rows)
+    assert_close(got[:, rows][:, :, hs], ref, torch.bfloat16, "orig full without kv_end (sampled)")
