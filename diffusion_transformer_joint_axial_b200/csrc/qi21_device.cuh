@@ -55,19 +55,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of the phase (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // try_wait with a suspend-time hint: a thread whose phase is not complete
 // sleeps (up to `ns` nanoseconds) instead of spinning, so waiting warps do not
 // take issue slots from the warps sharing their SMSP.
@@ -97,25 +84,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     // a 1 us suspend hint: measured as fast as or faster than 20 us on every
     // workload (a shorter sleep after the phase completes)
     if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (global_ns() - t0 > limit_ns) {
-      if (abort != nullptr) *abort = 1;
-      record_status(status, kStatusTimeout, where);
-      return false;
-    }
-  }
-}
-
-// The same bounded wait, polling without ever suspending: for the one warp
-// whose reaction time is on the critical path (the MMA issuer).
-__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, volatile int* abort,
-                                               uint32_t* status, uint32_t where,
-                                               uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (true) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_test_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
     if (global_ns() - t0 > limit_ns) {
       if (abort != nullptr) *abort = 1;
