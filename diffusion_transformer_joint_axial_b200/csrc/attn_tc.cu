@@ -137,9 +137,10 @@ struct __align__(1024) Smem {
   uint64_t q_full[2], q_rot[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_half[2], p_full[2], o_done[2], o_free[2];
-  // [unit parity][tile]: the epilogue drains one unit behind, so a tile whose
-  // unit has a single key tile can finish its softmax twice before the
-  // epilogue waits; one barrier per unit parity keeps the phases apart
+  // [item parity][tile]: the epilogue can fall an item behind (while it
+  // merges a split unit, say), and a tile with a single key tile can then
+  // finish its softmax twice before the epilogue waits; one barrier per item
+  // parity keeps the phases apart
   uint64_t l_ready[2][2];
   // [tile][epilogue warp]: bulk loads of the pieces to merge after a CTA's last item
   uint64_t mrg[2][4];
