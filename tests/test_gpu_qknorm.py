@@ -108,3 +108,28 @@ def test_qknorm_t2i_full_size_sampled(cuda_device):
     trows = rows[rows >= P] - P
     assert_close(g["oc"][:, trows][:, :, hs], g["o"][:, P + trows][:, :, hs].to(torch.float64).numpy(),
                  torch.bfloat16, "t2i qk-norm cached vs full target rows")
+
+
+def test_qknorm_cached_step_tail_split(cuda_device):
+    """The fused norm on a cached step whose last wave is split into 3
+    key-range pieces per unit (80 units of 48 key tiles on a 148-SM B200):
+    every target row of every head against the float64 oracle."""
+    segs = [T_(256), I_(32, 32, 1), I_(32, 32, 2), I_(32, 32, 3), I_(32, 32, 4), I_(24, 32, 5),
+            I_(32, 32, 0)]
+    L = sum(W.seg_tokens(s) for s in segs)
+    T = W.seg_tokens(segs[-1])
+    P = L - T
+    B, H = 1, 20
+    q, k, v = W.draw_qkv(B, L, H, 33, "bf16")
+    q, k = (q.float() * 6.0).to(torch.bfloat16), (k.float() * 0.2).to(torch.bfloat16)
+    wq, wk = W.qk_norm_weights()
+    qt, kt, vt = W.draw_qkv(B, T, H, 34, "bf16")
+    qt = (qt.float() * 3.0).to(torch.bfloat16)
+    g = _run(segs, q, k, v, P, wq, wk, cuda_device, qt, kt, vt)
+    pos, _ = O.positions(segs)
+    wq64, wk64 = W.as_f64(wq), W.as_f64(wk)
+    kn = O.rms_norm(W.as_f64(k), wk64, EPS)
+    okc, ovc = O.prefix_cache(kn, W.as_f64(v), pos, P)
+    refc = O.attn_cached(O.rms_norm(W.as_f64(qt), wq64, EPS), O.rms_norm(W.as_f64(kt), wk64, EPS),
+                         W.as_f64(vt), pos[P:], okc, ovc)
+    assert_close(g["oc"], refc, torch.bfloat16, "qk-norm cached step, tail split")
