@@ -93,3 +93,24 @@ def test_denoise_cache_reuse_bit_exact_on_tile_aligned_prefix(cuda_device):
         out.append(m.x.cpu())
     assert torch.equal(out[0], out[1])
     assert (out[0].float() - x0.float()).abs().mean() > 0.1
+
+
+def test_denoise_tail_split_against_oracle(cuda_device):
+    """The loop on a layout whose cached steps split their work units into 4
+    key-range pieces (2 heads x 3 query-tile pairs of 16 key tiles): against
+    the float64 oracle with the bounds above."""
+    segs = [W.text(256), W.image(32, 32, 1), W.image(24, 32, 0)]
+    sig = W.denoise_sigmas(STEPS)
+    params, draw = W.denoise_model(HEADS, CH, BLOCKS, STEPS, seed=41)
+    L = sum(W.seg_tokens(s) for s in segs)
+    T = W.seg_tokens(segs[-1])
+    x0, ph = draw(1, L - T, T, 42)
+    m = qi.denoise.DenoiseModel(segs, HEADS, CH, BLOCKS, STEPS, sig, device=cuda_device, cached=True)
+    m.load(params, x0, ph)
+    m.run()
+    m.check()
+    got = W.as_f64(m.x.cpu())
+    ref = O.denoise(W.as_f64(x0), W.as_f64(ph), _f64(params), segs, sig, cached=True)
+    err = np.abs(got - ref)
+    print("split layout, denoise vs oracle: max %.3g mean %.3g" % (err.max(), err.mean()))
+    assert err.max() <= 6e-2 and err.mean() <= 1e-2
