@@ -93,3 +93,55 @@ def test_tail_split_repeated_calls_on_one_workspace(cuda_device):
     ref = O.attn_cached(W.as_f64(qt.cpu()), W.as_f64(kt.cpu()), W.as_f64(vt.cpu()), pos[P:], okc, ovc)
     assert_close(outs[0], ref, torch.bfloat16, "repeated calls")
     assert np.isfinite(outs[0].float().numpy()).all()
+
+
+def _cached_vs_oracle(cuda_device, segs, B, H, seed, ws_bytes=None):
+    L = sum(W.seg_tokens(s) for s in segs)
+    T = W.seg_tokens(segs[-1])
+    P = L - T
+    q, k, v = W.draw_qkv(B, L, H, seed, "bf16")
+    pos, _ = O.positions(segs)
+    if P > 0:
+        g = gpu_full(segs, q, k, v, P)
+        kc, vc, pt = g["kc"], g["vc"], g["pos"][P:].contiguous()
+    else:
+        kc = vc = torch.zeros((B, H, 0, 128), dtype=torch.bfloat16, device=cuda_device)
+        pt, _ = qi.rope_positions(segs, cuda_device)
+    okc, ovc = O.prefix_cache(W.as_f64(k), W.as_f64(v), pos, P)
+    qt, kt, vt = W.draw_qkv(B, T, H, seed + 1, "bf16")
+    need = qi.cached_workspace_size(B, H, P, T, torch.bfloat16) if ws_bytes is None else ws_bytes
+    ws = qi.new_workspace(need, cuda_device)
+    oc = qi.attn_cached(qt.to(cuda_device), kt.to(cuda_device), vt.to(cuda_device), pt.to(cuda_device), kc, vc,
+                        workspace=ws)
+    assert qi.workspace_status(ws) == 0
+    ref = O.attn_cached(W.as_f64(qt), W.as_f64(kt), W.as_f64(vt), pos[P:], okc, ovc)
+    assert_close(oc.cpu(), ref, torch.bfloat16, "cached")
+    return oc.cpu()
+
+
+def test_tail_split_empty_prefix(cuda_device):
+    """P = 0: the keys are the target's own (48 units of 24 key tiles: 3 pieces)."""
+    assert split_pieces(48, 24) == 3
+    _cached_vs_oracle(cuda_device, [I_(48, 64, 0)], 1, 4, 51)
+
+
+def test_tail_split_partial_last_tile(cuda_device):
+    """T = 1000: the last query-tile pair has a full first tile and a second
+    tile of 104 rows; its unit is split like the others (12 units of 24 key
+    tiles: 4 pieces), and the padding rows are never stored."""
+    assert split_pieces(12, 24) == 4
+    _cached_vs_oracle(cuda_device, [T_(2000), I_(25, 40, 0)], 1, 3, 53)
+
+
+def test_tail_split_needs_no_scratch(cuda_device):
+    """A workspace holding only the position table and the rotated keys (no
+    split scratch) still runs, unsplit, with the same result up to rounding."""
+    segs = CASES["k3_prefix_5120"][0]
+    B, H = 1, 20
+    T = W.seg_tokens(segs[-1])
+    rnd = lambda x: (x + 255) // 256 * 256
+    minimum = rnd(rnd(256 + T * 64 * 8) + B * H * T * 128 * 2)
+    assert minimum < qi.cached_workspace_size(B, H, 5120, T, torch.bfloat16)
+    small = _cached_vs_oracle(cuda_device, segs, B, H, 55, ws_bytes=minimum)
+    split = _cached_vs_oracle(cuda_device, segs, B, H, 55)
+    assert (small.float() - split.float()).abs().max().item() < 2e-2
