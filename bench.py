@@ -723,12 +723,14 @@ def run_ours(args, world, rank, local):
                    "timing": "whole C-ABI calls (rotation/cache pre-pass + attention kernel), CUDA events "
                              "on the launch stream",
                    "qk_norm": bool(args.qk_norm),
+                   "k_rotation": args.k_rotation,
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "dp%d (independent requests per GPU)" % world},
         "full_step": hr["full_step"],
         "cached_step": hr["cached_step"],
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(head), "traffic_unit": "bytes/call",
+                     "frac": achieved / peak, "traffic": ncu_traffic(head) if args.k_rotation == "pre-pass" else None,
+                     "traffic_unit": "bytes/call",
                      "kernel": "attention calls of the step (full + cached): rotation/cache pre-pass + "
                                "qi21::tc::attn_tc_kernel",
                      "peak_kind": "%s bf16 dense burst (cuBLAS), MEASURED_PEAKS.json" % kind
@@ -759,7 +761,15 @@ def main(argv=None):
     ap.add_argument("--denoise-blocks", type=int, default=32)
     ap.add_argument("--qk-norm", action="store_true",
                     help="time the variant with the QK-RMSNorm fused in front of RoPE")
+    ap.add_argument("--k-rotation", default="pre-pass", choices=["pre-pass", "attention"],
+                    help="where the keys outside the Prefix cache are rotated: once per token in "
+                         "the pre-pass (default), or per key tile inside the attention kernel "
+                         "(an ablation, sets QI21_K_ROTATION)")
     args = ap.parse_args(argv)
+    if args.k_rotation == "attention":
+        os.environ["QI21_K_ROTATION"] = "attention"
+    else:
+        os.environ.pop("QI21_K_ROTATION", None)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup(args)

@@ -2,6 +2,7 @@
 // workspace carving, and the kernel sequence of each entry point.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -235,6 +236,18 @@ size_t qi21_attn_cached_workspace_size(int32_t B, int32_t H, int64_t P, int64_t 
   return base + split_bytes(B, H, T);
 }
 
+// Ablation of where the keys are rotated: QI21_K_ROTATION=attention (read on
+// every call) leaves the keys that do not go to the Prefix cache unrotated in
+// the pre-pass and has the tensor-core kernel rotate each of their tiles in
+// shared memory before its S MMAs.  bf16 calls without QK-RMSNorm only; such a
+// call runs without tail split.  Default: every key is rotated once, in the
+// pre-pass.
+static bool k_rotation_in_attention(qi21_dtype dt, const float* norm_k) {
+  if (dt != QI21_BF16 || norm_k != nullptr) return false;
+  const char* s = getenv("QI21_K_ROTATION");
+  return s != nullptr && strcmp(s, "attention") == 0;
+}
+
 static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi21_dtype dt,
                                   const void* q, const void* k, const void* v, const int32_t* pos,
                                   const int32_t* kv_end, void* o, void* k_cache, void* v_cache,
@@ -289,10 +302,14 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;
   rp.norm_eps = eps;
+  // the target's keys (past the cached Prefix) may be left to the attention kernel
+  const bool rot_k1 = cache && k_rotation_in_attention(dt, norm_k);
+  rp.k_rot_end = rot_k1 ? split : L;
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   // without a mask every unit costs the same, so the last wave may be split
-  if (dt == QI21_BF16 && kv_end == nullptr) carve_split(a, rp, ws, w.total, workspace_bytes, B, H, L);
+  if (dt == QI21_BF16 && kv_end == nullptr && !rot_k1)
+    carve_split(a, rp, ws, w.total, workspace_bytes, B, H, L);
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
@@ -308,8 +325,14 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   a.k0 = KvSource{rp.k_dst0, split, kHeadDim, split * kHeadDim, (int64_t)H * split * kHeadDim};
   a.k1 = KvSource{cache ? ws_k : nullptr, L - split, kHeadDim, (L - split) * kHeadDim,
                   (int64_t)H * (L - split) * kHeadDim};
-  // values straight from v (token-major), split the same way
   const size_t eb = elem_bytes(dt);
+  if (rot_k1) {
+    // raw target keys straight from k (token-major)
+    a.k1 = KvSource{static_cast<const uint8_t*>(k) + (size_t)split * tokstride * eb, L - split, tokstride,
+                    kHeadDim, L * tokstride};
+    a.rot_k1 = 1;
+  }
+  // values straight from v (token-major), split the same way
   a.v0 = KvSource{v, split, tokstride, kHeadDim, L * tokstride};
   a.v1 = KvSource{static_cast<const uint8_t*>(v) + (size_t)split * tokstride * eb, L - split, tokstride,
                   kHeadDim, L * tokstride};
@@ -367,12 +390,14 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   rp.omega = make_omega();
   rp.k_norm_w = norm_k;
   rp.norm_eps = eps;
+  const bool rot_k1 = k_rotation_in_attention(dt, norm_k);
+  rp.k_rot_end = rot_k1 ? 0 : T;
 
   // Tail-split scratch: whatever the workspace holds past the minimum layout
   // (none: the call runs unsplit).
   AttnArgs a;
   memset(&a, 0, sizeof(a));
-  if (dt == QI21_BF16) carve_split(a, rp, ws, w.total, workspace_bytes, B, H, T);
+  if (dt == QI21_BF16 && !rot_k1) carve_split(a, rp, ws, w.total, workspace_bytes, B, H, T);
   cudaError_t e = launch_rope_prep(rp, dt == QI21_F32, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope pre-pass launch");
 
@@ -386,6 +411,10 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   a.kv_end = nullptr;  // the target sees every key
   a.k0 = KvSource{k_cache, P, kHeadDim, P * kHeadDim, (int64_t)H * P * kHeadDim};
   a.k1 = KvSource{ws_k, T, kHeadDim, T * kHeadDim, (int64_t)H * T * kHeadDim};
+  if (rot_k1) {
+    a.k1 = KvSource{k, T, tokstride, kHeadDim, T * tokstride};  // raw target keys
+    a.rot_k1 = 1;
+  }
   a.v0 = KvSource{v_cache, P, kHeadDim, P * kHeadDim, (int64_t)H * P * kHeadDim};
   a.v1 = KvSource{v, T, tokstride, kHeadDim, T * tokstride};
   a.o = o;

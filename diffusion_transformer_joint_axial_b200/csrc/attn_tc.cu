@@ -107,6 +107,10 @@ struct Params {
   // split_k key-range pieces each, so num_items = head_units + (num_units -
   // head_units) * split_k.  split_k == 1: every item is a whole unit.
   int32_t head_units, split_k, num_items;
+  // 1: source-1 keys arrive unrotated and the epilogue warps rotate each of
+  // their tiles (row r of source 1 uses table row ktab1 + r) before the MMA
+  // warp may read it (k_rot); whole units only
+  int32_t rot_k1, ktab1;
   uint4* part;         // [slot][tile][4 row quarters][16 chunks][32 rows]: a piece's O / l, 8 bf16 per chunk
   float2* part_ml;     // [slot][tile][128 rows]: the piece's (row max, row sum)
   uint32_t* part_cnt;  // [tail unit][tile][4 row quarters]: pieces finished (zeroed by the pre-pass)
@@ -136,6 +140,7 @@ struct __align__(1024) Smem {
   int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
   uint64_t q_full[2], q_rot[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t k_rot[kStages];  // source-1 rotation done (rot_k1 only)
   uint64_t s_full[2], p_half[2], p_full[2], o_done[2], o_free[2];
   // [item parity][tile]: the epilogue can fall an item behind (while it
   // merges a split unit, say), and a tile with a single key tile can then
@@ -282,22 +287,50 @@ __device__ __forceinline__ void load_table_row(const uint4* cs, uint4 (&tb)[16])
   for (int i = 0; i < 16; ++i) tb[i] = __ldg(cs + i);
 }
 
+// One 16-byte chunk (four adjacent pairs (2m, 2m+1)) turned by its four
+// (cos, sin) fp16 pairs, rounded once to bf16.
+__device__ __forceinline__ void turn_chunk(uint4& x, const uint4& tb) {
+  const __half2* tc = reinterpret_cast<const __half2*>(&tb);
+  uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 xv = unpack_bf16x2(w[e]);
+    const float2 r = __half22float2(tc[e]);  // (cos, sin) of pair e of the chunk
+    w[e] = pack_bf16x2(fmaf(xv.x, r.x, -xv.y * r.y), fmaf(xv.x, r.y, xv.y * r.x));
+  }
+}
+// Chunk c of row t of a 128B-swizzled 128 x 128 tile (two 64-column halves).
+__device__ __forceinline__ uint4* tile_chunk(uint8_t* row, int c, int t) {
+  return reinterpret_cast<uint4*>(row + (c >> 3) * kHalfBytes + (((c & 7) ^ (t & 7)) << 4));
+}
+
 // Rotation of one query row in its 128B-swizzled tile (row t): each adjacent
 // pair (2m, 2m+1) turned by the token's (cos, sin), rounded once to bf16.
 __device__ __forceinline__ void rotate_q_row(uint8_t* qrow, const uint4 (&tb)[16], int t) {
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
-    uint4* ptr = reinterpret_cast<uint4*>(qrow + (c >> 3) * kHalfBytes + (((c & 7) ^ (t & 7)) << 4));
+    uint4* ptr = tile_chunk(qrow, c, t);
     uint4 x = *ptr;
-    const __half2* tc = reinterpret_cast<const __half2*>(&tb[c]);
-    uint32_t* w = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 xv = unpack_bf16x2(w[e]);
-      const float2 r = __half22float2(tc[e]);  // (cos, sin) of pair 4 c + e
-      w[e] = pack_bf16x2(fmaf(xv.x, r.x, -xv.y * r.y), fmaf(xv.x, r.y, xv.y * r.x));
-    }
+    turn_chunk(x, tb[c]);
     *ptr = x;
+  }
+}
+
+// The same for one row of an unrotated key tile, with the table read two
+// chunks at a time (the epilogue warps that do it run on 80 registers).
+__device__ __forceinline__ void rotate_k_row(uint8_t* krow, const uint4* cs, int t) {
+#pragma unroll
+  for (int c0 = 0; c0 < 16; c0 += 2) {
+    uint4 tb[2], x[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) tb[i] = __ldg(cs + c0 + i);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) x[i] = *tile_chunk(krow, c0 + i, t);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      turn_chunk(x[i], tb[i]);
+      *tile_chunk(krow, c0 + i, t) = x[i];
+    }
   }
 }
 
@@ -436,6 +469,50 @@ __device__ __forceinline__ float row_max_from(const float* sv, int c0, float (&m
   return fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), fmaxf(fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7])));
 }
 
+// O / l -> bf16 of one whole unit's tile, this warp's 32 rows, in two
+// 64-column halves.  Each warp stages its own rows in shared memory (128B-
+// swizzled, the TMA layout) and writes them with one TMA store (rows past Lq
+// are clipped; a box wholly past Lq is not issued).  O's TMEM columns are
+// released as soon as the second half has been read, long before the stores
+// finish.  No barrier spans warps, so a warp that gives up on a timed-out
+// wait cannot hold the others.
+__device__ __forceinline__ void store_tile(Smem& S, const Params& p, uint32_t tO, float inv,
+                                           uint8_t* stage, int lane, int s, int h, int b,
+                                           int row_first) {
+  for (int hh = 0; hh < 2; ++hh) {
+    if (lane == 0) bulk_wait_read_all();  // this warp's slice of the stage is free
+    __syncwarp();
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t orow[32];
+      tmem_ld32(tO + 64 * hh + 32 * c, orow);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
+                             __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
+        const int chunk = 4 * c + e;  // 16-byte chunk of the 128-byte row
+        *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    if (hh == 1) {
+      tc_fence_before();
+      mbar_arrive(smem_u32(&S.o_free[s]));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row_first < p.Lq) {
+      tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, h, row_first, b);
+      bulk_commit_group();
+    }
+    __syncwarp();
+  }
+}
+
 // Dynamic schedule: the K-producer warp takes the next unit from a global
 // counter (units are numbered in decreasing-cost order) and publishes it in a
 // shared-memory ring; every role reads the same sequence through next_unit().
@@ -538,6 +615,71 @@ __device__ __forceinline__ void piece_weights(const Params& p, int slot0, int s,
   for (int i = 0; i < kMaxSplit; ++i) a[i] *= inv;
 }
 
+// Epilogue warps of a call whose source-1 keys arrive unrotated (rot_k1):
+// besides draining O they rotate every source-1 key tile in place, one row
+// per thread from the query table, and arrive on k_rot for every key tile
+// (source 0 is already rotated), which the MMA warp waits on instead of
+// k_full.  An item's O is drained once the next item's first two key tiles
+// are done, so those are ready when the item's last P*V completes.  Whole
+// units only (the launcher does not split such a call).
+__device__ __forceinline__ void rotk1_epilogue(Smem& S, const Params& p, uint32_t tmem,
+                                               volatile int* abort_flag, int warp, int lane) {
+  const int t = threadIdx.x & 127;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  uint8_t* stage = S.ostage + (warp & 3) * 32 * 128;
+  uint32_t kc = 0, cnt[2] = {0, 0}, sc = 0;
+  bool ok = true, have_prev = false;
+  Unit prev = {};
+  auto drain = [&](const Unit& d) {
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (d.N[s] == 0) continue;
+      const uint32_t par = cnt[s] & 1u;
+      const uint32_t lpar = (cnt[s] >> 1) & 1u;
+      ++cnt[s];
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.l_ready[par][s]), lpar, abort_flag,
+                                            p.status, 0x440 | s));
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.o_done[s]), par, abort_flag,
+                                            p.status, 0x450 | s));
+      if (!ok) break;
+      tc_fence_after();
+      store_tile(S, p, tmem + lane_base + 256 + s * kHeadDim, 1.f / S.row_l[par][s][t], stage, lane,
+                 s, d.h, d.b, d.row0 + s * BM + (warp & 3) * 32);
+    }
+  };
+  while (ok) {
+    const int u = next_unit(S, p, sc, abort_flag, ok);
+    if (u < 0) break;
+    const Unit U = decode_item(p, u);
+    const int N = max(U.N[0], U.N[1]);
+    for (int n = 0; n < N && ok; ++n) {
+      const KTile kt = key_tile(p, U.kb + n);
+      const int st = kc % kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_full[st]), (kc / kStages) & 1u, abort_flag,
+                                            p.status, 0x430 | st));
+      if (!ok) break;
+      ++kc;
+      // rows past the source's end were zero-filled by the load: left alone
+      if (kt.src == 1 && kt.row + t < p.n1)
+        rotate_k_row(S.k[st] + t * 128, p.table + (size_t)(p.ktab1 + kt.row + t) * 16, t);
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&S.k_rot[st]));
+      if (have_prev && n == min(1, N - 1)) {
+        drain(prev);
+        have_prev = false;
+      }
+    }
+    if (!ok) break;
+    if (have_prev) drain(prev);  // an item without key tiles
+    prev = U;
+    have_prev = true;
+  }
+  if (ok && have_prev) drain(prev);
+}
+
+// kRotK1: source-1 keys arrive unrotated (Params::rot_k1); a separate
+// instantiation, so the default kernel carries none of its checks.
+template <bool kRotK1>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -563,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&S.k_full[s]), 1);
       mbar_init(smem_u32(&S.k_empty[s]), 1);
+      mbar_init(smem_u32(&S.k_rot[s]), BM);
       mbar_init(smem_u32(&S.v_full[s]), 1);
       mbar_init(smem_u32(&S.v_empty[s]), 1);
     }
@@ -701,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // prologue: S_s(0)
         {
           const int st = kc % kStages;
-          ok = wait(S.k_full[st], (kc / kStages) & 1u, 0x210);
+          ok = wait(kRotK1 ? S.k_rot[st] : S.k_full[st], (kc / kStages) & 1u, 0x210);
           if (!ok) break;
           tc_fence_after();
           const uint64_t kdesc = st ? kdesc1 : kdesc0;
@@ -759,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             if (n + 1 < U.N[s]) {
               if (!k_ready) {
-                ok = wait(S.k_full[kst], (kc / kStages) & 1u, 0x260 | kst);
+                ok = wait(kRotK1 ? S.k_rot[kst] : S.k_full[kst], (kc / kStages) & 1u, 0x260 | kst);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
@@ -799,6 +942,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     setmaxnreg_dec_epilogue();
     const int t = threadIdx.x & 127;  // row == TMEM lane (warp % 4 picks the lane quarter)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    if constexpr (kRotK1) {
+      rotk1_epilogue(S, p, tmem, abort_flag, warp, lane);
+    } else {
     uint32_t cnt[2] = {0, 0}, sc = 0;
     bool ok = true;
     int u = next_unit(S, p, sc, abort_flag, ok);
@@ -823,46 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint8_t* stage = S.ostage + (warp & 3) * 32 * 128;
         const int row_first = prev.row0 + s * BM + (warp & 3) * 32;
         if (prev.slot < 0) {
-          // O / l -> bf16 in two 64-column halves.  Each warp stages its own
-          // 32 rows in shared memory (128B-swizzled, the TMA layout) and
-          // writes them with one TMA store (rows past Lq are clipped; a box
-          // wholly past Lq is not issued).  O's TMEM columns are released as
-          // soon as the second half has been read, long before the stores
-          // finish.  No barrier spans warps, so a warp that gives up on a
-          // timed-out wait cannot hold the others.
-          const float inv = 1.f / S.row_l[par][s][t];
-          for (int hh = 0; hh < 2; ++hh) {
-            if (lane == 0) bulk_wait_read_all();  // this warp's slice of the stage is free
-            __syncwarp();
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              uint32_t orow[32];
-              tmem_ld32(tO + 64 * hh + 32 * c, orow);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  w[i] = pack_bf16x2(__uint_as_float(orow[8 * e + 2 * i]) * inv,
-                                     __uint_as_float(orow[8 * e + 2 * i + 1]) * inv);
-                const int chunk = 4 * c + e;  // 16-byte chunk of the 128-byte row
-                *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            }
-            if (hh == 1) {
-              tc_fence_before();
-              mbar_arrive(smem_u32(&S.o_free[s]));
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && row_first < p.Lq) {
-              tma_store_4d(&p.tm_o, smem_u32(stage), 64 * hh, prev.h, row_first, prev.b);
-              bulk_commit_group();
-            }
-            __syncwarp();
-          }
+          store_tile(S, p, tO, 1.f / S.row_l[par][s][t], stage, lane, s, prev.h, prev.b, row_first);
           continue;
         }
         // A piece of a split unit: its O / l (bf16) and (row max, row sum)
@@ -948,6 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         break;
       }
+    }
     }
     // the shared-memory stage must stay valid until the last stores read it
     if (lane == 0) bulk_wait_read_all();
@@ -1149,6 +1257,8 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.unit_counter = a.unit_counter;
   p.q_norm_w = a.q_norm_w;
   p.norm_eps = a.norm_eps;
+  p.rot_k1 = a.rot_k1;
+  p.ktab1 = (int32_t)(a.Lq - a.k1.n);
   // Tail split (unmasked calls, where every unit visits the same key tiles):
   // the r units of the last, partial wave go out as k pieces each when that
   // shortens the wave.  Costs in key tiles of one unit, from per-CTA
@@ -1159,7 +1269,7 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   // it measured 3 % slower).
   p.head_units = p.num_units;
   p.split_k = 1;
-  if (a.kv_end == nullptr && a.split_slots > 0 && num_sms > 0) {
+  if (a.kv_end == nullptr && a.split_slots > 0 && num_sms > 0 && !a.rot_k1) {
     const int r = p.num_units % num_sms;
     const int N = (p.n0 + tc::BN - 1) / tc::BN + (p.n1 + tc::BN - 1) / tc::BN;
     if (r > 0 && r <= a.split_cnt_units) {
@@ -1182,10 +1292,14 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   p.part_cnt = a.split_cnt;
   const size_t smem = sizeof(tc::Smem) + 1024;
   cudaError_t err =
-      cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(p.rot_k1 ? tc::attn_tc_kernel<true> : tc::attn_tc_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = p.num_items < num_sms ? p.num_items : num_sms;
-  tc::attn_tc_kernel<<<grid, tc::kThreads, smem, stream>>>(p);
+  if (p.rot_k1)
+    tc::attn_tc_kernel<true><<<grid, tc::kThreads, smem, stream>>>(p);
+  else
+    tc::attn_tc_kernel<false><<<grid, tc::kThreads, smem, stream>>>(p);
   note_launch();
   return cudaGetLastError();
 }

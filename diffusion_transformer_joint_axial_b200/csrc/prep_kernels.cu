@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int64_t tok = tok0 + t;
   const int H = p.H;
   const bool has_tok = tok < p.Lk;
+  const bool has_k = tok < p.k_rot_end && has_tok;  // this token's key is rotated here
   const int iters = (H + SPT - 1) / SPT;  // the same for every thread (shuffle reductions)
   if (blockIdx.x == 0 && blockIdx.y == 0) {
     if (p.unit_counter != nullptr && threadIdx.x == 0) *p.unit_counter = 0u;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(kPrepThreads)
 #pragma unroll
     for (int j = 0; j < kPrepHeadsInFlight; ++j) {
       const int h = h0 + (i0 + j) * SPT;
-      if (has_tok && i0 + j < iters && h < H) x[j] = ld_stream(kp + static_cast<int64_t>(h) * kHeadDim);
+      if (has_k && i0 + j < iters && h < H) x[j] = ld_stream(kp + static_cast<int64_t>(h) * kHeadDim);
     }
   };
   load_batch(0);
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kPrepThreads)
     for (int j = 0; j < kPrepHeadsInFlight; ++j) {
       if (i0 + j >= iters) break;
       const int h = h0 + (i0 + j) * SPT;
-      const bool live = has_tok && h < H;
+      const bool live = has_k && h < H;
       float rs = 1.f;
       if (norm) {
         // the row's CPR chunks are CPR consecutive lanes

@@ -66,6 +66,9 @@ struct RopePrepParams {
   Omega omega;
   const float* k_norm_w;   // [128] QK-RMSNorm weight of K, or null (no norm)
   float norm_eps;
+  // Keys of tokens [k_rot_end, Lk) are neither rotated nor written here (the
+  // attention kernel rotates them itself); Lk: every token's key is rotated.
+  int64_t k_rot_end;
 };
 cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream);
 
@@ -103,6 +106,10 @@ struct AttnArgs {
   void* split_part;   // split_slots x 2 tiles x 128 rows x 128 bf16
   void* split_ml;     // split_slots x 2 tiles x 128 rows x float2
   int32_t split_slots;
+  // 1: k1 holds the raw keys of the last k1.n query rows (token-major, not
+  // rotated), and the tensor-core kernel rotates each of their tiles in shared
+  // memory from the query table before its S MMAs (no tail split then).
+  int32_t rot_k1;
 };
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_sms);

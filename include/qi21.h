@@ -33,6 +33,15 @@
  *   per-token cos/sin table and the rotated keys of the call).  The paths
  *   that need no workspace are qi21_rope_positions and
  *   qi21_attn_cached_noalloc.
+ * - Key rotation placement (an ablation; the result is the same up to
+ *   rounding): by default every key is rotated once, by the call's pre-pass.
+ *   With the environment variable QI21_K_ROTATION=attention (read on every
+ *   call) a QI21_BF16 call without QK-RMSNorm leaves the keys that do not go
+ *   to the Prefix cache unrotated, and the attention kernel rotates each of
+ *   their tiles in shared memory (from the fp16 query table) before it reads
+ *   them, once per query-tile pair that visits the tile; such a call does not
+ *   split its last wave.  The Prefix keys stored in the cache are rotated by
+ *   the pre-pass either way.
  */
 #ifndef QI21_H
 #define QI21_H
