@@ -1262,7 +1262,7 @@ cudaError_t launch_attn_tc_bf16(const AttnArgs& a, cudaStream_t stream, int num_
   // Tail split (unmasked calls, where every unit visits the same key tiles):
   // the r units of the last, partial wave go out as k pieces each when that
   // shortens the wave.  Costs in key tiles of one unit, from per-CTA
-  // timelines: each item start (Q load and rotation, the first tiles' fill)
+  // timelines: each item (the pipeline's fill and drain around its key tiles)
   // about 3.5; the merge the last CTA cannot overlap, plus the slowdown of
   // the whole units running beside the pieces, about 9 (with these the
   // 384-unit 1024^2 step, 34 key tiles per unit, stays unsplit: split into 3
