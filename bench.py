@@ -42,12 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # pre-pass plus the attention kernel -- from one ncu capture of each kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum), per workload.  Valid only for
 # the kernel sources they were taken on: any other source reports null.
-NCU_TRAFFIC = {"sources_sha256": "1d1b71d10647a9bb",
+NCU_TRAFFIC = {"sources_sha256": "dc2bdfdab6c1700a",
                # mean of the full and the cached call
-               "bytes_per_call": {"t2i": ((28.399e6 + 0.056e6 + 82.097e6 + 2.271e6)
-                                          + (25.250e6 + 0.000e6 + 79.905e6 + 1.373e6)) / 2,
-                                  "hires": ((315.192e6 + 262.544e6 + 2583.854e6 + 277.286e6)
-                                            + (201.720e6 + 144.773e6 + 2403.676e6 + 234.570e6)) / 2}}
+               "bytes_per_call": {"t2i": ((28.400e6 + 0.056e6 + 82.174e6 + 3.304e6)
+                                          + (25.250e6 + 0.000e6 + 79.890e6 + 1.996e6)) / 2,
+                                  "hires": ((315.114e6 + 262.664e6 + 2608.485e6 + 277.106e6)
+                                            + (201.688e6 + 144.887e6 + 2429.671e6 + 234.787e6)) / 2}}
 
 
 def kernel_sources_digest(read=None):

@@ -9,12 +9,12 @@ binding: it marshals torch tensors into that ABI and nothing else.
 from ._binding import (HEAD_DIM, LIB_PATH, QI21Error, Segment, alloc_cache, attn_cached, attn_full,
                        cached_workspace_size, full_workspace_size, interleave_gate_up, launch_count, linear,
                        linear_residual, linear_swiglu,
-                       load_library, new_workspace, rmsnorm, rope_positions,
+                       load_library, new_workspace, rmsnorm, rope_positions, rope_table, rope_table_size,
                        selftest_wait_timeout, swiglu, workspace_status)
 from . import denoise
 from .steploop import DenoiseLoop
 
 __all__ = ["DenoiseLoop", "HEAD_DIM", "LIB_PATH", "QI21Error", "Segment", "alloc_cache", "attn_cached",
            "attn_full", "cached_workspace_size", "full_workspace_size", "interleave_gate_up", "launch_count",
-           "linear", "linear_residual", "linear_swiglu", "load_library", "new_workspace", "rmsnorm", "rope_positions",
+           "linear", "linear_residual", "linear_swiglu", "load_library", "new_workspace", "rmsnorm", "rope_positions", "rope_table", "rope_table_size",
            "selftest_wait_timeout", "swiglu", "workspace_status"]

@@ -30,6 +30,8 @@ EXPORTED = (
     "qi21_attn_full_workspace_size", "qi21_attn_full", "qi21_attn_full_qknorm",
     "qi21_attn_cached_workspace_size", "qi21_attn_cached", "qi21_attn_cached_qknorm",
     "qi21_attn_cached_noalloc",
+    # the request's rotation table and the cached step that reads it
+    "qi21_rope_table_size", "qi21_rope_table", "qi21_attn_cached_tabled",
     # projections and the rest of a block of the denoising loop
     "qi21_linear", "qi21_linear_residual", "qi21_linear_swiglu", "qi21_rmsnorm", "qi21_swiglu",
     # status, errors, counters, timing and self-tests
@@ -101,6 +103,13 @@ def load_library(path=LIB_PATH):
     L.qi21_attn_cached_noalloc.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                            _vp, _vp]
     L.qi21_attn_cached_noalloc.restype = _i32
+    L.qi21_rope_table_size.argtypes = [_i64]
+    L.qi21_rope_table_size.restype = _sz
+    L.qi21_rope_table.argtypes = [_vp, _i64, _vp, _sz, _vp]
+    L.qi21_rope_table.restype = _i32
+    L.qi21_attn_cached_tabled.argtypes = [_i32, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _sz, _vp]
+    L.qi21_attn_cached_tabled.restype = _i32
     for name in ("qi21_rope_positions", "qi21_attn_full", "qi21_attn_cached", "qi21_attn_full_qknorm",
                  "qi21_attn_cached_qknorm", "qi21_workspace_status", "qi21_selftest_wait_timeout"):
         getattr(L, name).restype = _i32
@@ -255,12 +264,37 @@ def attn_full(q, k, v, pos, kv_end, prefix_len, k_cache=None, v_cache=None, out=
     return out
 
 
-def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk_norm=None):
+def rope_table_size(n):
+    """Bytes of the rotation table of n tokens."""
+    return int(load_library().qi21_rope_table_size(n))
+
+
+def rope_table(pos, out=None):
+    """The rotation table of the tokens whose positions are ``pos`` ([n, 3]
+    int32 on the device): built once per request, read by every later step
+    (``attn_cached(..., rope_table=t)``).  Returns a uint8 device tensor
+    (``out``, if given: ``rope_table_size(n)`` bytes)."""
+    L_ = _cuda_lib()
+    dev = pos.device
+    n = pos.shape[0]
+    _need(pos, "pos", (n, 3), torch.int32, dev)
+    table = out
+    if table is None:
+        table = torch.empty(int(L_.qi21_rope_table_size(n)), dtype=torch.uint8, device=dev)
+    _need(table, "out", (int(L_.qi21_rope_table_size(n)),), torch.uint8, dev)
+    with torch.cuda.device(dev):
+        _check(L_.qi21_rope_table(_ptr(pos), n, _ptr(table), table.numel(), _stream(dev)))
+    return table
+
+
+def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk_norm=None, rope_table=None):
     """Later step: target queries over [cached prefix K/V || fresh target K/V], no mask.
 
     q, k, v: [B, T, H, 128]; pos_tgt [T, 3]; k_cache, v_cache [B, H, P, 128].
     ``qk_norm`` as for :func:`attn_full` (the cache must come from a full step
-    with the same norm).
+    with the same norm).  ``rope_table``: the target's table from
+    :func:`rope_table` (then ``pos_tgt`` may be None), read instead of
+    computing the angles again; not with ``qk_norm``.
     """
     L_ = _cuda_lib()
     B, T, H, D = q.shape
@@ -268,7 +302,12 @@ def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk
     code = _dtype_code(q)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, (B, T, H, HEAD_DIM), dt, dev)
-    _need(pos_tgt, "pos_tgt", (T, 3), torch.int32, dev)
+    if rope_table is None:
+        _need(pos_tgt, "pos_tgt", (T, 3), torch.int32, dev)
+    else:
+        if qk_norm is not None:
+            raise ValueError("rope_table is not taken together with qk_norm")
+        _need(rope_table, "rope_table", (int(L_.qi21_rope_table_size(T)),), torch.uint8, dev)
     P = k_cache.shape[2]
     _need(k_cache, "k_cache", (B, H, P, HEAD_DIM), dt, dev)
     _need(v_cache, "v_cache", (B, H, P, HEAD_DIM), dt, dev)
@@ -280,7 +319,11 @@ def attn_cached(q, k, v, pos_tgt, k_cache, v_cache, out=None, workspace=None, qk
         workspace = new_workspace(need, dev)
     norm = _norm_args(qk_norm, dev)
     with torch.cuda.device(dev):
-        if norm is None:
+        if rope_table is not None:
+            _check(L_.qi21_attn_cached_tabled(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(rope_table),
+                                              _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(dev)))
+        elif norm is None:
             _check(L_.qi21_attn_cached(B, H, P, T, code, _ptr(q), _ptr(k), _ptr(v), _ptr(pos_tgt),
                                        _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(dev)))

@@ -343,11 +343,15 @@ static qi21_status attn_full_impl(int32_t B, int32_t H, int64_t L, int64_t P, qi
   return run_attention(a, dt, st);
 }
 
+// rope_table: the target's table from qi21_rope_table (its float32 pairs feed
+// the pre-pass's key rotation, its float16 pairs the queries' rotation), or
+// null: computed here from pos_tgt.
 static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
                                     const void* q, const void* k, const void* v,
                                     const int32_t* pos_tgt, const void* k_cache, const void* v_cache,
                                     void* o, const float* norm_q, const float* norm_k, float eps,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
+                                    void* workspace, size_t workspace_bytes, void* stream,
+                                    const void* rope_table = nullptr) {
   QI21_TRY(check_common(B, H, dt));
   if (P < 0 || T < 0 || P > (int64_t)1 << 30 || T > (int64_t)1 << 30)
     return fail(QI21_ERR_INVALID_ARG, "P and T must be in [0, 2^30] (P=%lld, T=%lld)", (long long)P, (long long)T);
@@ -356,7 +360,10 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   QI21_TRY(check_ptr(k, "k"));
   QI21_TRY(check_ptr(v, "v"));
   QI21_TRY(check_ptr(o, "o"));
-  QI21_TRY(check_ptr(pos_tgt, "pos_tgt"));
+  if (rope_table == nullptr)
+    QI21_TRY(check_ptr(pos_tgt, "pos_tgt"));
+  else
+    QI21_TRY(check_ptr(rope_table, "rope_table"));
   if (P > 0) {
     QI21_TRY(check_ptr(k_cache, "k_cache"));
     QI21_TRY(check_ptr(v_cache, "v_cache"));
@@ -392,6 +399,15 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   rp.norm_eps = eps;
   const bool rot_k1 = k_rotation_in_attention(dt, norm_k);
   rp.k_rot_end = rot_k1 ? 0 : T;
+  // a given table: the pre-pass reads its float32 pairs, the attention its
+  // float16 (bf16 path) or float32 pairs; the workspace's table is not written
+  const void* table_t16 = nullptr;
+  if (rope_table != nullptr) {
+    rp.pos = nullptr;
+    rp.table_in = rope_table;
+    rp.table = nullptr;
+    table_t16 = static_cast<const uint8_t*>(rope_table) + (size_t)T * kPairs * sizeof(float2);
+  }
 
   // Tail-split scratch: whatever the workspace holds past the minimum layout
   // (none: the call runs unsplit).
@@ -407,7 +423,8 @@ static qi21_status attn_cached_impl(int32_t B, int32_t H, int64_t P, int64_t T, 
   a.H = H;
   a.Lq = T;
   a.q = q;
-  a.table = table;
+  a.table = rope_table == nullptr ? static_cast<const void*>(table)
+                                  : (dt == QI21_BF16 ? table_t16 : rope_table);
   a.kv_end = nullptr;  // the target sees every key
   a.k0 = KvSource{k_cache, P, kHeadDim, P * kHeadDim, (int64_t)H * P * kHeadDim};
   a.k1 = KvSource{ws_k, T, kHeadDim, T * kHeadDim, (int64_t)H * T * kHeadDim};
@@ -449,6 +466,37 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
                              void* stream) {
   return attn_cached_impl(B, H, P, T, dt, q, k, v, pos_tgt, k_cache, v_cache, o, nullptr, nullptr,
                           0.f, workspace, workspace_bytes, stream);
+}
+
+size_t qi21_rope_table_size(int64_t n) {
+  if (n < 0) return 0;
+  return (size_t)n * kPairs * (sizeof(float2) + sizeof(uint32_t));
+}
+
+qi21_status qi21_rope_table(const int32_t* pos, int64_t n, void* table, size_t table_bytes, void* stream) {
+  if (n < 0 || n > (int64_t)1 << 30) return fail(QI21_ERR_INVALID_ARG, "n out of range (%lld)", (long long)n);
+  if (n == 0) return QI21_OK;
+  QI21_TRY(check_ptr(pos, "pos"));
+  QI21_TRY(check_ptr(table, "table"));
+  if (table_bytes < qi21_rope_table_size(n))
+    return fail(QI21_ERR_INVALID_ARG, "table too small: %zu < %zu bytes", table_bytes, qi21_rope_table_size(n));
+  RopeTableParams p;
+  p.pos = pos;
+  p.n = n;
+  p.t32 = table;
+  p.t16 = static_cast<uint8_t*>(table) + (size_t)n * kPairs * sizeof(float2);
+  p.omega = make_omega();
+  const cudaError_t e = launch_rope_table(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotation table launch");
+  return QI21_OK;
+}
+
+qi21_status qi21_attn_cached_tabled(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                    const void* q, const void* k, const void* v, const void* rope_table,
+                                    const void* k_cache, const void* v_cache, void* o, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return attn_cached_impl(B, H, P, T, dt, q, k, v, nullptr, k_cache, v_cache, o, nullptr, nullptr, 0.f,
+                          workspace, workspace_bytes, stream, rope_table);
 }
 
 qi21_status qi21_attn_cached_qknorm(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,

@@ -76,6 +76,13 @@ Omega make_omega() {
   return o;
 }
 
+// (cos, sin) of pair m of a token at (f, h, w) = pos[0..2], in float64.
+__device__ __forceinline__ void pair_sincos(const int32_t* pos, int m, const Omega& om, double& c,
+                                            double& s) {
+  const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
+  sincos(static_cast<double>(pos[axis]) * om.w[m], &s, &c);
+}
+
 constexpr int kPrepTokens = 4;  // tokens per CTA
 constexpr int kPrepThreads = 256;
 
@@ -202,11 +209,11 @@ __global__ void __launch_bounds__(kPrepThreads)
   if (norm && threadIdx.x < kHeadDim) wn[threadIdx.x] = p.k_norm_w[threadIdx.x];
   if (threadIdx.x < kPrepTokens * kPairs) {
     const int tt = threadIdx.x / kPairs, m = threadIdx.x % kPairs;
-    if (tok0 + tt < p.Lk) {
-      const int axis = m < kBandPairs0 ? 0 : (m < kBandPairs01 ? 1 : 2);
-      const double ang = static_cast<double>(p.pos[3 * (tok0 + tt) + axis]) * p.omega.w[m];
+    if (tok0 + tt < p.Lk && p.table_in != nullptr) {
+      cs[tt][m] = static_cast<const float2*>(p.table_in)[(tok0 + tt) * kPairs + m];
+    } else if (tok0 + tt < p.Lk) {
       double sd, cd;
-      sincos(ang, &sd, &cd);
+      pair_sincos(p.pos + 3 * (tok0 + tt), m, p.omega, cd, sd);
       const float2 v = make_float2(static_cast<float>(cd), static_cast<float>(sd));
       cs[tt][m] = v;
       if (p.table != nullptr && b == 0) {
@@ -280,6 +287,29 @@ cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t str
     rope_prep_kernel<float><<<grid, kPrepThreads, 0, stream>>>(p);
   else
     rope_prep_kernel<__nv_bfloat16><<<grid, kPrepThreads, 0, stream>>>(p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// ======================================================= rotation table ==
+// One thread per (token, pair): the pre-pass's float64 angle, rounded once to
+// fp32 and once to fp16.
+__global__ void rope_table_kernel(const __grid_constant__ RopeTableParams p) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i >= p.n * kPairs) return;
+  const int64_t tok = i / kPairs;
+  const int m = static_cast<int>(i - tok * kPairs);
+  double sd, cd;
+  pair_sincos(p.pos + 3 * tok, m, p.omega, cd, sd);
+  static_cast<float2*>(p.t32)[i] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+  static_cast<__half2*>(p.t16)[i] = __halves2half2(__double2half(cd), __double2half(sd));
+}
+
+cudaError_t launch_rope_table(const RopeTableParams& p, cudaStream_t stream) {
+  if (p.n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (p.n * kPairs + threads - 1) / threads;
+  rope_table_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
   note_launch();
   return cudaGetLastError();
 }

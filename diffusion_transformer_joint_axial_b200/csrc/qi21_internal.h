@@ -69,8 +69,23 @@ struct RopePrepParams {
   // Keys of tokens [k_rot_end, Lk) are neither rotated nor written here (the
   // attention kernel rotates them itself); Lk: every token's key is rotated.
   int64_t k_rot_end;
+  // [Lk][64] float2 (cos, sin) built earlier by the table kernel (pos is then
+  // not read and no angle is computed), or null
+  const void* table_in;
 };
 cudaError_t launch_rope_prep(const RopePrepParams& p, bool f32, cudaStream_t stream);
+
+// A request's rotation table: per token its 64 (cos, sin) pairs, float2 in
+// t32 [n][64] and rounded to half2 in t16 [n][64], the same values the
+// pre-pass computes.
+struct RopeTableParams {
+  const int32_t* pos;  // [n][3]
+  int64_t n;
+  void* t32;
+  void* t16;
+  Omega omega;
+};
+cudaError_t launch_rope_table(const RopeTableParams& p, cudaStream_t stream);
 
 // --------------------------------------------------------------- attention
 // One key/value source: rows of one (batch, head) are `row` elements apart,

@@ -197,6 +197,35 @@ qi21_status qi21_attn_cached(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dt
                              void* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qi21_rope_table -- a request's rotation table: for each of n tokens the 64
+ * (cos, sin) pairs of its axial angles pos * theta^(-2i/d_axis), computed in
+ * float64 ("3A - 3D Axial RoPE (16, 56, 56)", section 1), stored rounded to
+ * float32 ([n][64] float2, first) and to float16 ([n][64] half2, after it).
+ * The target's positions do not change over the denoising steps, so the
+ * table of its T tokens can be built once per request and handed to every
+ * later step's qi21_attn_cached_tabled, whose pre-pass then computes no
+ * angles; the result is bit-identical to qi21_attn_cached with the same
+ * positions.
+ *   pos     device [n][3] int32 (qi21_rope_positions' rows of those tokens).
+ *   table   device, at least qi21_rope_table_size(n) bytes, 16-byte aligned;
+ *           written (caller-owned; valid as long as the caller keeps it).
+ * Returns QI21_ERR_INVALID_ARG for a bad size or pointer or a short buffer.
+ */
+size_t qi21_rope_table_size(int64_t n);
+qi21_status qi21_rope_table(const int32_t* pos, int64_t n, void* table, size_t table_bytes, void* stream);
+
+/*
+ * qi21_attn_cached_tabled -- qi21_attn_cached with the target's rotation
+ * table given (rope_table: device, qi21_rope_table of the T target tokens)
+ * instead of its positions.  Every other argument, the workspace size and the
+ * errors are those of qi21_attn_cached.
+ */
+qi21_status qi21_attn_cached_tabled(int32_t B, int32_t H, int64_t P, int64_t T, qi21_dtype dt,
+                                    const void* q, const void* k, const void* v, const void* rope_table,
+                                    const void* k_cache, const void* v_cache, void* o, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * qi21_attn_full_qknorm / qi21_attn_cached_qknorm -- the same two steps with
  * the QK-RMSNorm that precedes RoPE fused in (overview card 4A "Single-Stream
  * DiT Attention & QK-RMSNorm"; close reading section 6: norm_q and norm_k are
