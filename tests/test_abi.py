@@ -214,3 +214,26 @@ def test_binding_fails_loudly_without_cuda(monkeypatch):
     monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
     with pytest.raises(qb.QI21Error):
         qb.rope_positions([{"kind": "text", "n": 4}])
+
+
+def test_rope_table_sizes_and_rejects(lib):
+    """qi21_rope_table: n x 64 pairs as float2 then half2 (12 bytes a pair);
+    bad sizes, pointers and short buffers are rejected before anything is
+    enqueued, and so are the tabled cached step's."""
+    p = ctypes.c_void_p
+    bad = qb.QI21_ERR_INVALID_ARG
+    for n in (0, 1, 77, 4096):
+        assert lib.qi21_rope_table_size(n) == n * 64 * 12
+    assert lib.qi21_rope_table_size(-1) == 0
+    tab = lambda n=16, pos=16, t=256, tb=16 * 768: lib.qi21_rope_table(
+        p(pos) if pos else None, n, p(t) if t else None, tb, None)
+    assert tab(n=-1) == bad and tab(n=(1 << 30) + 1) == bad
+    assert tab(pos=None) == bad and tab(pos=20) == bad       # NULL / misaligned positions
+    assert tab(t=None) == bad and tab(t=24) == bad           # NULL / misaligned table
+    assert tab(tb=16 * 768 - 16) == bad                      # table buffer too small
+    assert tab(n=0, pos=None, t=None) == qb.QI21_OK          # nothing to do
+    cached = lambda T=16, table=16: lib.qi21_attn_cached_tabled(
+        1, 2, 16, T, qb.QI21_BF16, p(16), p(16), p(16), p(table) if table else None, p(16), p(16), p(16),
+        p(256), 1 << 30, None)
+    assert cached(T=-1) == bad
+    assert cached(table=None) == bad and cached(table=24) == bad
