@@ -42,12 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # pre-pass plus the attention kernel -- from one ncu capture of each kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum), per workload.  Valid only for
 # the kernel sources they were taken on: any other source reports null.
-NCU_TRAFFIC = {"sources_sha256": "dc2bdfdab6c1700a",
+NCU_TRAFFIC = {"sources_sha256": "d9e77a0f51985532",
                # mean of the full and the cached call
-               "bytes_per_call": {"t2i": ((28.400e6 + 0.056e6 + 82.174e6 + 3.304e6)
-                                          + (25.250e6 + 0.000e6 + 79.890e6 + 1.996e6)) / 2,
-                                  "hires": ((315.114e6 + 262.664e6 + 2608.485e6 + 277.106e6)
-                                            + (201.688e6 + 144.887e6 + 2429.671e6 + 234.787e6)) / 2}}
+               "bytes_per_call": {"t2i": ((28.399e6 + 0.098e6 + 82.082e6 + 2.291e6)
+                                          + (25.250e6 + 0.000e6 + 79.879e6 + 1.046e6)) / 2,
+                                  "hires": ((315.112e6 + 262.514e6 + 2569.402e6 + 276.766e6)
+                                            + (201.684e6 + 144.807e6 + 2396.354e6 + 231.838e6)) / 2}}
 
 
 def kernel_sources_digest(read=None):

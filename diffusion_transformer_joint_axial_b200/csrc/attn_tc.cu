@@ -32,10 +32,15 @@
 //   warps 8-11  epilogue, 80 regs: drains each item's O (O / l -> bf16 ->
 //               TMA store, or a piece's partial result and the merge) as soon
 //               as its MMAs are done
-//   warp  12    TMA producer of Q tiles and the K ring (2 stages), 112 regs
+//   warp  12    TMA producer of Q tiles and of the key tiles, 112 regs
 //   warp  13    TMEM allocator and tcgen05.mma issuer, 112 regs
-//   warp  14    TMA producer of the V ring (2 stages), 112 regs
+//   warp  14    TMA producer of the value tiles, 112 regs
 //   warp  15    idle, 112 regs
+// Key and value tiles share a two-slot ring: slot t holds key tile t and
+// value tile t - 1 (numbered over the CTA's whole sequence of items), the two
+// tiles one step of the MMA warp reads, so each step waits on one barrier
+// and releases one (a unit's last slot, whose key tile is the next unit's
+// first, is released after that unit's first S MMAs).
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the upper 64 columns of its S and is the A
 // operand of the P*V MMA, so P never touches shared memory.  P is released in
@@ -139,7 +144,10 @@ struct __align__(1024) Smem {
   alignas(16) float qnw[kHeadDim];  // QK-RMSNorm weight of Q (when given)
   int32_t sched_unit[kSchedSlots];  // units handed out by the K producer (-1: none left)
   uint64_t q_full[2], q_rot[2], q_empty[2];
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  // ring slot t holds key tile t and value tile t - 1 (global indices, in
+  // stage t % kStages); full: both producers' loads landed, empty: the MMA
+  // warp has read both tiles
+  uint64_t slot_full[kStages], slot_empty[kStages];
   uint64_t k_rot[kStages];  // source-1 rotation done (rot_k1 only)
   uint64_t s_full[2], p_half[2], p_full[2], o_done[2], o_free[2];
   // [item parity][tile]: the epilogue can fall an item behind (while it
@@ -618,8 +626,8 @@ __device__ __forceinline__ void piece_weights(const Params& p, int slot0, int s,
 // Epilogue warps of a call whose source-1 keys arrive unrotated (rot_k1):
 // besides draining O they rotate every source-1 key tile in place, one row
 // per thread from the query table, and arrive on k_rot for every key tile
-// (source 0 is already rotated), which the MMA warp waits on instead of
-// k_full.  An item's O is drained once the next item's first two key tiles
+// (source 0 is already rotated), which the MMA warp waits on as well as on
+// the slot.  An item's O is drained once the next item's first two key tiles
 // are done, so those are ready when the item's last P*V completes.  Whole
 // units only (the launcher does not split such a call).
 __device__ __forceinline__ void rotk1_epilogue(Smem& S, const Params& p, uint32_t tmem,
@@ -655,7 +663,7 @@ __device__ __forceinline__ void rotk1_epilogue(Smem& S, const Params& p, uint32_
     for (int n = 0; n < N && ok; ++n) {
       const KTile kt = key_tile(p, U.kb + n);
       const int st = kc % kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_full[st]), (kc / kStages) & 1u, abort_flag,
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.slot_full[st]), (kc / kStages) & 1u, abort_flag,
                                             p.status, 0x430 | st));
       if (!ok) break;
       ++kc;
@@ -703,11 +711,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int w = 0; w < 4; ++w) mbar_init(smem_u32(&S.mrg[s][w]), 1);
     }
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&S.k_full[s]), 1);
-      mbar_init(smem_u32(&S.k_empty[s]), 1);
+      mbar_init(smem_u32(&S.slot_full[s]), 2);  // the K and the V producer
+      mbar_init(smem_u32(&S.slot_empty[s]), 1);
       mbar_init(smem_u32(&S.k_rot[s]), BM);
-      mbar_init(smem_u32(&S.v_full[s]), 1);
-      mbar_init(smem_u32(&S.v_empty[s]), 1);
     }
     for (int s = 0; s < kSchedSlots; ++s) {
       mbar_init(smem_u32(&S.sched_full[s]), 1);
@@ -741,8 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     setmaxnreg_dec_other();
     if (warp == kWarpLoad || warp == kWarpLoadV) {
       // --------------------------------------------------------- producers
-      // Warp 12 loads Q and K, warp 14 loads V, so a wait for a free V stage
-      // never holds back the next K tile (and the other way round).
+      // Warp 12 loads Q and the key tiles, warp 14 the value tiles; both
+      // count into the slot's barrier.
       const bool do_qk = warp == kWarpLoad;
       uint32_t sc = 0;
       // The whole warp runs the loop (every value is warp-uniform, so the
@@ -750,6 +756,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const bool leader = elect_one_sync();
       uint32_t kc = 0, vc = 0, ql[2] = {0, 0}, qi[2] = {0, 0};
       bool ok = true;
+      // Ring slot t holds key tile t and value tile t - 1 (global indices):
+      // the MMA warp uses both in the same step, and one barrier counts both
+      // producers.  Slot 0 has no value tile: the V producer arrives alone.
+      if (!do_qk && leader) mbar_arrive(smem_u32(&S.slot_full[0]));
+      __syncwarp();
       while (ok) {
         if (do_qk) publish_unit(S, p, sc, leader, abort_flag, ok);
         const int u = next_unit(S, p, sc, abort_flag, ok);
@@ -775,23 +786,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const KTile t = key_tile(p, U.kb + n);
           if (do_qk) {
             const int st = kc % kStages;
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.k_empty[st]), ((kc / kStages) & 1u) ^ 1u,
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.slot_empty[st]), ((kc / kStages) & 1u) ^ 1u,
                                                   abort_flag, p.status, 0x110 | st));
             if (!ok) break;
             if (leader) {
-              const uint32_t bar = smem_u32(&S.k_full[st]);
+              const uint32_t bar = smem_u32(&S.slot_full[st]);
               mbar_arrive_expect_tx(bar, kTileBytes);
               load_kv_tile(t.src ? &p.tm_k1 : &p.tm_k0, t.src ? p.k1_tok : p.k0_tok,
                            smem_u32(S.k[st]), bar, t.row, U.h, U.b);
             }
             ++kc;
           } else {
-            const int st = vc % kStages;
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.v_empty[st]), ((vc / kStages) & 1u) ^ 1u,
+            const uint32_t slot = vc + 1;
+            const int st = slot % kStages;
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.slot_empty[st]), ((slot / kStages) & 1u) ^ 1u,
                                                   abort_flag, p.status, 0x120 | st));
             if (!ok) break;
             if (leader) {
-              const uint32_t bar = smem_u32(&S.v_full[st]);
+              const uint32_t bar = smem_u32(&S.slot_full[st]);
               mbar_arrive_expect_tx(bar, kTileBytes);
               load_kv_tile(t.src ? &p.tm_v1 : &p.tm_v0, t.src ? p.v1_tok : p.v0_tok,
                            smem_u32(S.v[st]), bar, t.row, U.h, U.b);
@@ -800,19 +812,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       }
+      // The last slot holds the last value tile and no key tile.
+      if (ok && do_qk) {
+        const int st = kc % kStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S.slot_empty[st]), ((kc / kStages) & 1u) ^ 1u,
+                                              abort_flag, p.status, 0x130 | st));
+        if (ok && leader) mbar_arrive(smem_u32(&S.slot_full[st]));
+        __syncwarp();
+      }
       // Every load this warp issued lands before the CTA may exit: wait
       // (bounded) for the last load issued into each stage.
       if (!ok) {
         for (int s = 0; s < 2 && do_qk; ++s)
           if (qi[s] > 0) mbar_wait(smem_u32(&S.q_full[s]), (qi[s] - 1) & 1u, nullptr, nullptr, 0);
         for (uint32_t st = 0; st < kStages; ++st) {
-          if (kc > st) {
+          if (kc > st && do_qk) {
             const uint32_t last = ((kc - 1 - st) / kStages) * kStages + st;
-            mbar_wait(smem_u32(&S.k_full[st]), (last / kStages) & 1u, nullptr, nullptr, 0);
+            mbar_wait(smem_u32(&S.slot_full[st]), (last / kStages) & 1u, nullptr, nullptr, 0);
           }
-          if (vc > st) {
-            const uint32_t last = ((vc - 1 - st) / kStages) * kStages + st;
-            mbar_wait(smem_u32(&S.v_full[st]), (last / kStages) & 1u, nullptr, nullptr, 0);
+          if (!do_qk && vc >= 1) {  // value tiles sit in slots 1 .. vc
+            const int last = (((int)vc - (int)st) / kStages) * kStages + (int)st;
+            if (last >= 1 && last <= (int)vc)
+              mbar_wait(smem_u32(&S.slot_full[st]), ((uint32_t)last / kStages) & 1u, nullptr, nullptr, 0);
           }
         }
       }
@@ -831,8 +852,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint64_t vdesc1 = sw128_desc(smem_u32(S.v[1]), kHalfBytes, 1024);
       uint32_t kc = 0, vc = 0, qv[2] = {0, 0}, ph[2] = {0, 0}, pf[2] = {0, 0}, of[2] = {0, 0};
       bool ok = true;
-      auto wait = [&](uint64_t& bar, uint32_t parity, uint32_t where) {
-        return __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar), parity, abort_flag, p.status, where));
+      auto wait = [&](uint64_t& bar, uint32_t parity, uint32_t where) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar), parity, abort_flag, p.status, where)) != 0;
+      };
+      // ring slot t (key tile t, value tile t - 1): slots below `waited` are full
+      uint32_t waited = 0;
+      auto need_slot = [&](uint32_t t, uint32_t where) -> bool {
+        if (t < waited) return true;
+        waited = t + 1;
+        return wait(S.slot_full[t % kStages], (t / kStages) & 1u, where | (t % kStages));
       };
       uint32_t sc = 0;
       while (ok) {
@@ -844,7 +872,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // prologue: S_s(0)
         {
           const int st = kc % kStages;
-          ok = wait(kRotK1 ? S.k_rot[st] : S.k_full[st], (kc / kStages) & 1u, 0x210);
+          ok = need_slot(kc, 0x210);
+          if (ok && kRotK1) ok = wait(S.k_rot[st], (kc / kStages) & 1u, 0x214);
           if (!ok) break;
           tc_fence_after();
           const uint64_t kdesc = st ? kdesc1 : kdesc0;
@@ -862,13 +891,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             __syncwarp();
           }
           if (!ok) break;
-          if (leader) mma_commit(smem_u32(&S.k_empty[st]));
+          if (leader) mma_commit(smem_u32(&S.slot_empty[st]));  // slot kc: both its tiles are read
           __syncwarp();
           ++kc;
         }
         for (int n = 0; n < N && ok; ++n) {
-          const int vst = vc % kStages;
-          ok = wait(S.v_full[vst], (vc / kStages) & 1u, 0x230 | vst);
+          const int vst = (vc + 1) % kStages;  // value tile vc sits in slot vc + 1
+          ok = need_slot(vc + 1, 0x230);
           if (!ok) break;
           tc_fence_after();
           const uint64_t vdesc = vst ? vdesc1 : vdesc0;
@@ -902,7 +931,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             if (n + 1 < U.N[s]) {
               if (!k_ready) {
-                ok = wait(kRotK1 ? S.k_rot[kst] : S.k_full[kst], (kc / kStages) & 1u, 0x260 | kst);
+                // key tile kc is in the slot already waited for (kc == vc + 1)
+                if (kRotK1) ok = wait(S.k_rot[kst], (kc / kStages) & 1u, 0x260 | kst);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
@@ -916,10 +946,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
           }
           if (!ok) break;
-          if (leader) {
-            mma_commit(smem_u32(&S.v_empty[vst]));
-            if (k_ready) mma_commit(smem_u32(&S.k_empty[kst]));
-          }
+          // slot vc + 1 is free once its key tile is read too: now, or (the
+          // unit's last step) after the next unit's first S MMAs
+          if (leader && k_ready) mma_commit(smem_u32(&S.slot_empty[vst]));
           __syncwarp();
           ++vc;
           if (k_ready) ++kc;
